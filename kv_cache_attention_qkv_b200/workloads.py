@@ -1,0 +1,209 @@
+"""Seeded synthetic inputs for one Flash-Cache step.
+
+This module only draws random numbers and lays them out; it holds none of the
+step's arithmetic, so both the CPU oracle and the CUDA path can be fed from it.
+
+Five workloads are defined, named by what they are:
+
+* ``tiny_fp32``      B=1, hidden 32, 2 heads x 16, theta 1e4, cache 64, fp32.
+                     Window at 40..43, 4 tracked positions drawn from 0..39.
+* ``layer_b1``       B=1, hidden 4096, 32 heads x 128, theta 5e5, cache 768
+                     (256 prompt + 512 generated), 64 tracked + 64 window, bf16.
+* ``batch32_uniform`` B=32, same layer, cache 1536 (1024 + 512) per sequence,
+                     64 tracked + 64 window, bf16.  The headline workload.
+* ``batch32_varlen`` B=32, same layer, cache length U[600, 2048] per sequence,
+                     window 16 or 64 and tracking budget 48/64/80 per sequence.
+* ``small_varlen``   a few-second ragged case for element-wise parity: B=3,
+                     hidden 256, 4 heads x 128, caches of 129..700 rows.
+
+The shapes follow LLaDA-8B (the model the Flash-dLLM pages evaluate); weights
+and caches are random, there is no dataset and no checkpoint.
+
+Every bf16 tensor is drawn in fp32 and rounded to bf16 by torch; the fp32 copy
+returned alongside holds exactly the bf16 values, so both sides start from the
+same numbers.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, List, Optional
+
+import numpy as np
+
+WORKLOADS = ("tiny_fp32", "layer_b1", "batch32_uniform", "batch32_varlen", "small_varlen")
+
+
+@dataclasses.dataclass
+class StepInputs:
+    """One step's inputs.  Float arrays are fp32 numpy holding dtype-exact values."""
+
+    name: str
+    dtype: str  # "bf16" or "fp32"
+    hidden: int
+    n_heads: int
+    head_dim: int
+    rope_theta: float
+    x: np.ndarray  # [T, hidden]
+    w_qkv: np.ndarray  # [3*H*d, hidden]; rows = [Q heads | K heads | V heads]
+    k_cache: np.ndarray  # [S, H, d] (prior contents)
+    v_cache: np.ndarray  # [S, H, d]
+    q_pos: np.ndarray  # int32 [T], absolute positions inside each sequence
+    cu_seqlens_q: np.ndarray  # int32 [B+1]
+    cu_seqlens_k: np.ndarray  # int32 [B+1]
+    cand_lo: np.ndarray  # int32 [B], candidate positions for reselection
+    cand_hi: np.ndarray  # int32 [B]
+    topk: np.ndarray  # int32 [B], tracking budget per sequence
+    window_start: np.ndarray  # int32 [B]
+    window_len: np.ndarray  # int32 [B]
+
+    @property
+    def batch(self) -> int:
+        return int(self.cu_seqlens_q.shape[0] - 1)
+
+    @property
+    def total_q(self) -> int:
+        return int(self.cu_seqlens_q[-1])
+
+    @property
+    def total_k(self) -> int:
+        return int(self.cu_seqlens_k[-1])
+
+    @property
+    def max_topk(self) -> int:
+        return int(self.topk.max())
+
+    def seq_slice_q(self, b: int) -> slice:
+        return slice(int(self.cu_seqlens_q[b]), int(self.cu_seqlens_q[b + 1]))
+
+    def seq_slice_k(self, b: int) -> slice:
+        return slice(int(self.cu_seqlens_k[b]), int(self.cu_seqlens_k[b + 1]))
+
+
+def to_bf16_exact(a: np.ndarray) -> np.ndarray:
+    """Round fp32 values to bf16 with torch and return them widened to fp32."""
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return t.to(torch.bfloat16).to(torch.float32).numpy()
+
+
+def _normal(rng: np.random.Generator, shape, std: float) -> np.ndarray:
+    a = rng.standard_normal(size=shape, dtype=np.float32)
+    if std != 1.0:
+        a *= np.float32(std)
+    return a
+
+
+def _layout(rng, lens_k: List[int], windows: List[int], budgets: List[int],
+            window_starts: List[int]):
+    """Query = tracked positions (ascending) then the masked window (ascending)."""
+    pos_rows = []
+    for L, w, kb, ws in zip(lens_k, windows, budgets, window_starts):
+        assert kb <= ws and ws + w <= L
+        tracked = np.sort(rng.choice(ws, size=kb, replace=False)).astype(np.int32)
+        window = np.arange(ws, ws + w, dtype=np.int32)
+        pos_rows.append(np.concatenate([tracked, window]))
+    n = [len(p) for p in pos_rows]
+    cu_q = np.zeros(len(n) + 1, np.int32)
+    cu_q[1:] = np.cumsum(n)
+    cu_k = np.zeros(len(lens_k) + 1, np.int32)
+    cu_k[1:] = np.cumsum(lens_k)
+    return np.concatenate(pos_rows).astype(np.int32), cu_q, cu_k
+
+
+def generate(name: str, seed: Optional[int] = None, batch: Optional[int] = None) -> StepInputs:
+    """Draw the named workload.  ``seed`` defaults to the workload's index.
+
+    ``batch`` overrides the number of sequences (used to draw a sub-sample or a
+    per-rank shard of the same recipe); per-sequence draws keep their recipe.
+    """
+    if name not in WORKLOADS:
+        raise ValueError(f"unknown workload {name!r}; known: {WORKLOADS}")
+    if seed is None:
+        seed = WORKLOADS.index(name)
+    rng = np.random.default_rng(seed)
+
+    if name == "tiny_fp32":
+        dtype, D, H, d, theta, w_std = "fp32", 32, 2, 16, 1.0e4, 0.1
+        B = batch or 1
+        lens = [64] * B
+        windows = [4] * B
+        budgets = [4] * B
+        starts = [40] * B
+    elif name == "layer_b1":
+        dtype, D, H, d, theta, w_std = "bf16", 4096, 32, 128, 5.0e5, 0.02
+        B = batch or 1
+        lens = [768] * B
+        windows = [64] * B
+        budgets = [64] * B
+        # 64-aligned window inside the generated span [256, 768)
+        starts = [int(256 + 64 * rng.integers(0, (768 - 256) // 64)) for _ in range(B)]
+    elif name == "batch32_uniform":
+        dtype, D, H, d, theta, w_std = "bf16", 4096, 32, 128, 5.0e5, 0.02
+        B = batch or 32
+        lens = [1536] * B
+        windows = [64] * B
+        budgets = [64] * B
+        starts = [int(1024 + 64 * rng.integers(0, (1536 - 1024) // 64)) for _ in range(B)]
+    elif name == "batch32_varlen":
+        dtype, D, H, d, theta, w_std = "bf16", 4096, 32, 128, 5.0e5, 0.02
+        B = batch or 32
+        lens = [int(v) for v in rng.integers(600, 2049, size=B)]
+        windows = [int(v) for v in rng.choice([16, 64], size=B)]
+        budgets = [int(v) for v in rng.choice([48, 64, 80], size=B)]
+        starts = []
+        for L, w, kb in zip(lens, windows, budgets):
+            lo = L - min(512, L - kb)
+            first = -(-lo // w) * w
+            last = L - w
+            starts.append(int(first + w * rng.integers(0, (last - first) // w + 1)))
+    else:  # small_varlen
+        dtype, D, H, d, theta, w_std = "bf16", 256, 4, 128, 5.0e5, 0.0625
+        B = batch or 3
+        base_lens = [700, 129, 333]
+        lens = [base_lens[i % 3] for i in range(B)]
+        windows = [64, 16, 64]
+        windows = [windows[i % 3] for i in range(B)]
+        budgets = [80, 48, 100]
+        budgets = [budgets[i % 3] for i in range(B)]
+        starts = []
+        for L, w, kb in zip(lens, windows, budgets):
+            first = -(-kb // w) * w
+            starts.append(int(first + w * rng.integers(0, (L - w - first) // w + 1)))
+
+    q_pos, cu_q, cu_k = _layout(rng, lens, windows, budgets, starts)
+    T, S = int(cu_q[-1]), int(cu_k[-1])
+
+    x = _normal(rng, (T, D), 1.0)
+    w = _normal(rng, (3 * H * d, D), w_std)
+    kc = _normal(rng, (S, H, d), 1.0)
+    vc = _normal(rng, (S, H, d), 1.0)
+    if dtype == "bf16":
+        x, w, kc, vc = (to_bf16_exact(a) for a in (x, w, kc, vc))
+
+    starts_a = np.asarray(starts, np.int32)
+    return StepInputs(
+        name=name, dtype=dtype, hidden=D, n_heads=H, head_dim=d, rope_theta=float(theta),
+        x=x, w_qkv=w, k_cache=kc, v_cache=vc, q_pos=q_pos,
+        cu_seqlens_q=cu_q, cu_seqlens_k=cu_k,
+        cand_lo=np.zeros(B, np.int32), cand_hi=starts_a.copy(),
+        topk=np.asarray(budgets, np.int32), window_start=starts_a,
+        window_len=np.asarray(windows, np.int32),
+    )
+
+
+def describe(name: str) -> Dict[str, object]:
+    """Shape summary of a workload without drawing its tensors."""
+    table = {
+        "tiny_fp32": dict(dtype="fp32", B=1, hidden=32, heads=2, head_dim=16, cache="64",
+                          query="4 tracked + 4 window"),
+        "layer_b1": dict(dtype="bf16", B=1, hidden=4096, heads=32, head_dim=128, cache="768",
+                         query="64 tracked + 64 window"),
+        "batch32_uniform": dict(dtype="bf16", B=32, hidden=4096, heads=32, head_dim=128,
+                                cache="1536", query="64 tracked + 64 window"),
+        "batch32_varlen": dict(dtype="bf16", B=32, hidden=4096, heads=32, head_dim=128,
+                               cache="U[600,2048]", query="48/64/80 tracked + 16/64 window"),
+        "small_varlen": dict(dtype="bf16", B=3, hidden=256, heads=4, head_dim=128,
+                             cache="700,129,333", query="80+64, 48+16, 100+64"),
+    }
+    return table[name]
