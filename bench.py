@@ -1,0 +1,392 @@
+"""Throughput of the Flash-Cache step on B200: query-tokens/s per fused step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one fc_step (QKV projection + RoPE + KV-cache write, bidirectional
+attention with importance, importance finalisation) plus one fc_topk_tracked
+on the headline workload: B=32 sequences, cache 1536 each, 128 query rows
+(64 tracked + 64 masked window) per sequence, hidden 4096, 32 heads x 128,
+bf16 (LLaDA-8B-shaped, random weights, synthetic data).
+
+Timing: W untimed warm-up steps, then K steps timed with CUDA events on the
+launching stream; an L2 flush (a 256 MiB write) runs between steps outside the
+events.  Under torchrun every rank runs its own batch (sequences are
+independent, no collective on the data path): value = all ranks' query tokens
+/ the slowest rank's time.  ``--impl reference`` times the fp64 CPU oracle on
+the host cores instead (the deliberately slow baseline arm).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "query-tokens/s per fused Flash-Cache step (B=32, L=1536); % of roofline"
+UNIT = "query-tokens/s"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def _work(inp):
+    """Algorithmic FLOPs and bytes of one step (what the method must compute/move)."""
+    T, S, D, H, d = inp.total_q, inp.total_k, inp.hidden, inp.n_heads, inp.head_dim
+    es = 2 if inp.dtype == "bf16" else 4
+    n = np.diff(inp.cu_seqlens_q).astype(np.int64)
+    L = np.diff(inp.cu_seqlens_k).astype(np.int64)
+    qkv_flops = 2.0 * T * D * 3 * H * d
+    attn_flops = 4.0 * H * d * float((n * L).sum())
+    qkv_bytes = es * (T * D + 3 * H * d * D) + es * 2 * T * H * d  # X, W read; K/V rows written
+    attn_bytes = es * 2 * S * H * d + es * T * H * d  # whole cache read, O written
+    return {"qkv_flops": qkv_flops, "attn_flops": attn_flops, "qkv_bytes": qkv_bytes,
+            "attn_bytes": attn_bytes, "flops": qkv_flops + attn_flops,
+            "bytes": qkv_bytes + attn_bytes}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None, "samples": len(rows), "reasons": reasons}
+
+
+def _dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from kv_cache_attention_qkv_b200 import FlashCache, workloads
+
+    ws, rank, local = _dist_env()
+    if ws > 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    # every rank draws its own batch of the same recipe
+    inp = workloads.generate(args.workload, seed=workloads.WORKLOADS.index(args.workload) + 1000 * rank)
+    dt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
+    f = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dtype=dt)
+    i = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+    x, w, kc, vc = f(inp.x), f(inp.w_qkv), f(inp.k_cache), f(inp.v_cache)
+    qp, cq, ck = i(inp.q_pos), i(inp.cu_seqlens_q), i(inp.cu_seqlens_k)
+    lo, hi, kps = i(inp.cand_lo), i(inp.cand_hi), i(inp.topk)
+    T, S, H, d, B = inp.total_q, inp.total_k, inp.n_heads, inp.head_dim, inp.batch
+    K = int(inp.topk.max())
+    layer = FlashCache(w, hidden=inp.hidden, n_heads=H, head_dim=d, rope_theta=inp.rope_theta,
+                       max_batch=B, max_total_q=T, max_total_k=S,
+                       max_seqlen_q=int(np.diff(inp.cu_seqlens_q).max()),
+                       max_pos=int(np.diff(inp.cu_seqlens_k).max()), max_topk=K)
+    out = torch.empty((T, H, d), device=dev, dtype=dt)
+    imp = torch.empty((S,), device=dev, dtype=torch.float32)
+    tracked = torch.empty((B, K), device=dev, dtype=torch.int32)
+    flush = torch.empty(256 * 1024 * 1024 // 4, device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.step(x, qp, cq, ck, kc, vc, out, imp)
+        n = layer.last_launch_count
+        layer.topk_tracked(imp, ck, lo, hi, K, tracked, k_per_seq=kps)
+        return n + layer.last_launch_count
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    if layer.get_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    launches = 0
+    layer.profile(True)
+    layer.profile_read()
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for k in range(args.steps):
+            flush.fill_(float(k))
+            ev[k][0].record(stream)
+            launches += step()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    per_kernel = layer.profile_read()
+    layer.profile(False)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = float(sum(step_ms))
+    err = layer.get_error()
+    if ws > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # ---- end to end through the public API with host buffers
+    x_h = torch.from_numpy(np.ascontiguousarray(inp.x)).to(dt).pin_memory()
+    small_h = {n: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).pin_memory()
+               for n, a in (("q_pos", inp.q_pos), ("cu_q", inp.cu_seqlens_q), ("cu_k", inp.cu_seqlens_k),
+                            ("lo", inp.cand_lo), ("hi", inp.cand_hi), ("kps", inp.topk))}
+    out_h = torch.empty((T, H, d), dtype=dt).pin_memory()
+    tr_h = torch.empty((B, K), dtype=torch.int32).pin_memory()
+    x_d = torch.empty_like(x)
+    small_d = {n: torch.empty_like(t, device=dev) for n, t in small_h.items()}
+    h2d = x_h.numel() * x_h.element_size() + sum(t.numel() * 4 for t in small_h.values())
+    d2h = out_h.numel() * out_h.element_size() + tr_h.numel() * 4
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        for n, t in small_h.items():
+            small_d[n].copy_(t, non_blocking=True)
+        layer.step(x_d, small_d["q_pos"], small_d["cu_q"], small_d["cu_k"], kc, vc, out, imp)
+        layer.topk_tracked(imp, small_d["cu_k"], small_d["lo"], small_d["hi"], K, tracked,
+                           k_per_seq=small_d["kps"])
+        out_h.copy_(out, non_blocking=True)
+        tr_h.copy_(tracked, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if ws > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    result = None
+    if rank == 0:
+        peaks = _peaks()
+        wk = _work(inp)
+        ms_per_step = total_ms / args.steps
+        tokens = T * ws * args.steps
+        value = tokens / (total_ms / 1e3)
+        # dominant kernel by measured share
+        names = {"qkv_rope_scatter": ("tensor", wk["qkv_flops"]), "attention": ("hbm", wk["attn_bytes"])}
+        dom = max(names, key=lambda k: per_kernel[k][0])
+        ms_k, n_k = per_kernel[dom]
+        avg_s = ms_k / max(n_k, 1) / 1e3
+        bound, work = names[dom]
+        if bound == "tensor":
+            achieved = work / avg_s / 1e12
+            peak = peaks["bf16_tflops"]
+            unit = "TFLOP/s"
+        else:
+            achieved = work / avg_s / 1e9
+            peak = peaks["hbm_gbs"]
+            unit = "GB/s"
+        t_roof = max(wk["flops"] / (peaks["bf16_tflops"] * 1e12), wk["bytes"] / (peaks["hbm_gbs"] * 1e9))
+        result = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": inp.dtype, "data": "synthetic",
+            "config": {"workload": args.workload, "batch": B, "seq_len": int(np.diff(inp.cu_seqlens_k).max()),
+                       "query_rows_per_seq": int(np.diff(inp.cu_seqlens_q).max()), "hidden": inp.hidden,
+                       "heads": H, "head_dim": d, "topk": K, "total_q": T, "total_k": S,
+                       "l2": "flushed between steps (256 MiB write)", "parallelism": f"sequence-sharded x{ws}"},
+            "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst)"},
+            "step_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": ms_per_step * 1e3,
+                              "frac": t_roof / (ms_per_step / 1e3), "flops": wk["flops"], "bytes": wk["bytes"]},
+            "kernels_ms_per_step": {k: v[0] / max(v[1], 1) for k, v in per_kernel.items()},
+            "gpu_launches": launches,
+            "device_error_word": err,
+            "e2e": {"value": T * ws * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+            "clocks": clk.summary(),
+        }
+        result["cpu_baseline"] = cpu_baseline(inp, budget_s=args.cpu_budget) if args.cpu_budget > 0 else None
+    layer.close()
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [p.get("num_threads") for p in threadpool_info() if p.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(inp, budget_s: float = 12.0):
+    """Time the fp64 oracle, as it stands, on a bounded sample of sequences."""
+    sys.path.insert(0, ROOT)
+    import oracle
+
+    done, tokens, t0 = 0, 0, time.perf_counter()
+    while True:
+        b = done % inp.batch
+        qs, ks = inp.seq_slice_q(b), inp.seq_slice_k(b)
+        r = oracle.step_sequence(inp.x[qs], inp.w_qkv, inp.q_pos[qs], inp.k_cache[ks], inp.v_cache[ks],
+                                 inp.n_heads, inp.head_dim, inp.rope_theta, inp.dtype)
+        imp = np.zeros(inp.total_k)
+        imp[ks] = r["importance"]
+        oracle.topk_tracked(imp, inp.cu_seqlens_k, inp.cand_lo, inp.cand_hi, inp.topk, int(inp.topk.max()))
+        done += 1
+        tokens += qs.stop - qs.start
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    return {"value": tokens / el, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+            "sample": f"{done} sequence(s) of workload {inp.name} ({tokens} query rows), "
+                      f"fp64 NumPy, {el:.1f} s wall"}
+
+
+def run_reference(args):
+    ws, rank, _ = _dist_env()
+    if rank != 0:
+        return None
+    from kv_cache_attention_qkv_b200 import workloads
+    import oracle
+
+    inp = workloads.generate(args.workload)
+    per_step = []
+    tokens_total = 0
+
+    def one(bidx):
+        qs, ks = inp.seq_slice_q(bidx), inp.seq_slice_k(bidx)
+        r = oracle.step_sequence(inp.x[qs], inp.w_qkv, inp.q_pos[qs], inp.k_cache[ks], inp.v_cache[ks],
+                                 inp.n_heads, inp.head_dim, inp.rope_theta, inp.dtype)
+        imp = np.zeros(inp.total_k)
+        imp[ks] = r["importance"]
+        oracle.topk_tracked(imp, inp.cu_seqlens_k, inp.cand_lo, inp.cand_hi, inp.topk, int(inp.topk.max()))
+        return qs.stop - qs.start
+
+    for k in range(args.warmup):
+        one(k % inp.batch)
+    for k in range(args.steps):
+        t0 = time.perf_counter()
+        tokens_total += one(k % inp.batch)
+        per_step.append(time.perf_counter() - t0)
+    el = sum(per_step)
+    value = tokens_total / el
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "sample_per_step": "one sequence (its query rows)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+                         "sample": f"{args.steps} sequence(s) of workload {args.workload}, one per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="batch32_uniform")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0,
+                    help="seconds of oracle time for cpu_baseline (0 = skip)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    res = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

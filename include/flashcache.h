@@ -1,0 +1,205 @@
+/*
+ * flashcache.h — C ABI of the B200 (sm_100a) Flash-Cache step.
+ *
+ * One Flash-Cache step (Flash-dLLM; paper-digest page, Fig. 2 caption, and the
+ * infernews post "Flash-dLLM: IO-aware KV caching and parallel decoding",
+ * Flash-Cache paragraph): every sequence b of a batch brings a query of n_b
+ * positions (the tracked positions plus the current masked window).  The step
+ *   1. projects the query rows x_r to q, k, v with W_qkv (no bias),
+ *   2. rotates q and k by RoPE at the rows' absolute positions,
+ *   3. writes k and v into the sequence's KV cache at those positions,
+ *   4. lets the query attend bidirectionally to the sequence's whole cache,
+ *   5. sums the attention probabilities of every key over heads and query rows
+ *      ("attention importance"),
+ * and a separate call (fc_topk_tracked) reselects, per sequence, the k
+ * candidate positions of highest importance as the next tracked set.
+ *
+ * Readings where the pages say nothing (the library follows them exactly):
+ *   - RoPE pairs element i with i + d/2 (rotate-half), angle pos*theta^(-2i/d);
+ *   - scores are q.k/sqrt(d); no biases; K/V heads = Q heads;
+ *   - the cache rows are written before attending, so the query sees its own
+ *     fresh K/V; every cache row of the sequence is attended (no mask);
+ *   - importance of key j = sum over heads and query rows of P[row, j];
+ *   - reselection ranks candidates by importance descending, then position
+ *     ascending.
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "dev" are CUDA device pointers on the handle's device;
+ *     pointers marked "host" are host memory.  The caller owns all of them and
+ *     keeps them alive until the work queued on the stream has finished.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Calls only enqueue work; none synchronises, except
+ *     fc_get_error.
+ *   - Integers are int32, floats IEEE binary32, bf16 values are raw 16-bit
+ *     bfloat16 patterns.  Every array is dense, row-major, without padding.
+ *   - A non-FC_OK status means nothing was enqueued, except FC_ERR_CUDA from a
+ *     launch, after which the stream's state is whatever CUDA reports.
+ *   - Problems only the device can see (a position outside its sequence, the
+ *     same position twice in one sequence, inconsistent cu_seqlens, a bad
+ *     candidate range, a barrier that timed out) set bits of a sticky device
+ *     error word, read and cleared by fc_get_error.  The offending rows or
+ *     sequences are skipped, no memory outside the documented arrays is
+ *     touched, and the step's results are then undefined.
+ */
+#ifndef FLASHCACHE_H
+#define FLASHCACHE_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FC_API __attribute__((visibility("default")))
+#else
+#define FC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fc_status {
+  FC_OK = 0,
+  FC_ERR_INVALID_ARG = -1,   /* a host-visible argument is wrong; nothing ran     */
+  FC_ERR_UNSUPPORTED = -2,   /* valid request outside what this build supports    */
+  FC_ERR_CUDA = -3,          /* a CUDA runtime/driver call failed                  */
+  FC_ERR_OOM = -4,           /* device allocation of the workspace failed          */
+  FC_ERR_DEVICE_CHECK = -5,  /* fc_get_error: the device error word is non-zero    */
+  FC_ERR_TIMEOUT = -6        /* fc_get_error: a kernel gave up on a barrier wait   */
+} fc_status;
+
+/* Element type of x, W_qkv, the KV cache and `out`. */
+enum { FC_DTYPE_BF16 = 0, FC_DTYPE_FP32 = 1 };
+
+/* Bits of the device error word (fc_get_error). */
+#define FC_DEVERR_POS_RANGE 0x01 /* q_pos[r] < 0 or >= its sequence's cache length */
+#define FC_DEVERR_POS_DUP 0x02   /* a position appears twice in one sequence       */
+#define FC_DEVERR_SEQLENS 0x04   /* cu_seqlens not monotone / totals disagree, or a
+                                    sequence longer than the configured limits      */
+#define FC_DEVERR_CAND 0x08      /* cand_lo/cand_hi/k_per_seq outside their ranges  */
+#define FC_DEVERR_TIMEOUT 0x10   /* a kernel abandoned a bounded barrier wait       */
+
+/* Model dimensions and capacity limits, fixed at fc_create. */
+typedef struct fc_config {
+  int hidden;        /* D: width of a query row x_r                                */
+  int n_heads;       /* H: attention heads (K/V heads are the same H)             */
+  int head_dim;      /* d: even; 128 selects the tensor-core path for bf16        */
+  double rope_theta; /* RoPE base theta (> 1)                                     */
+  int dtype;         /* FC_DTYPE_BF16 or FC_DTYPE_FP32                            */
+  int max_batch;     /* largest B a step may pass (<= 4096)                       */
+  int max_total_q;   /* largest T = sum n_b                                       */
+  int max_total_k;   /* largest S = sum L_b                                       */
+  int max_seqlen_q;  /* largest n_b                                               */
+  int max_pos;       /* largest cache length L_b (L_b <= max_pos <= 262144)       */
+  int max_topk;      /* largest k of fc_topk_tracked (<= 1024)                    */
+} fc_config;
+
+typedef struct fc_handle fc_handle;
+
+/*
+ * fc_create — validate `cfg`, bind the projection weights and allocate the
+ * handle's workspace on the current CUDA device.
+ *   cfg    host; copied.
+ *   w_qkv  dev, [3*H*d, D] of cfg->dtype, row-major (each output row is K-major,
+ *          i.e. contiguous along D).  Rows 0..H*d-1 are the Q heads, then the K
+ *          heads, then the V heads; head h occupies rows h*d..h*d+d-1 of its
+ *          block.  Kept by pointer: the caller keeps it alive and unchanged
+ *          until fc_destroy.  16-byte aligned.
+ *   out    host; receives the handle.
+ * Returns FC_ERR_INVALID_ARG for a NULL pointer or an inconsistent config,
+ * FC_ERR_UNSUPPORTED for a config this build cannot run, FC_ERR_OOM /
+ * FC_ERR_CUDA if the workspace cannot be set up (no device, out of memory).
+ * Synchronous (it uploads the RoPE table).
+ */
+FC_API fc_status fc_create(const fc_config* cfg, const void* w_qkv, fc_handle** out);
+
+/*
+ * fc_step — one Flash-Cache step on a packed, variable-length batch.
+ *   batch         B >= 1, <= max_batch.
+ *   x             dev, [T, D] of dtype: query rows of all sequences, sequence
+ *                 b in rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1.
+ *   q_pos         dev, int32 [T]: absolute position of every query row inside
+ *                 its sequence, 0 <= q_pos[r] < L_b, distinct within a sequence.
+ *   cu_seqlens_q  dev, int32 [B+1]: 0 = cu[0] <= cu[1] <= ... <= cu[B] = T.
+ *   cu_seqlens_k  dev, int32 [B+1]: the same over cache rows, cu[B] = S;
+ *                 L_b = cu_seqlens_k[b+1] - cu_seqlens_k[b] <= max_pos.
+ *   total_q       T (host int), <= max_total_q.  With T = 0 nothing is
+ *                 written except `importance` (zeroed when accumulate = 0).
+ *   total_k       S (host int), <= max_total_k.
+ *   k_cache       dev, [S, H, d] of dtype, updated in place: row
+ *   v_cache       cu_seqlens_k[b] + q_pos[r] receives the rotated k (resp. v)
+ *                 of query row r, rounded to nearest-even in dtype.  All other
+ *                 rows are only read.  16-byte aligned.
+ *   out           dev, [T, H, d] of dtype: attention output of every query row.
+ *   importance    dev, float [S] or NULL (then not computed).  Per key j of
+ *                 sequence b: sum over heads and query rows of b of the
+ *                 normalised attention probability of j.  With accumulate = 0
+ *                 it is overwritten, with accumulate = 1 the step's values are
+ *                 added to what it holds (e.g. to sum over layers).
+ * Host-detectable errors return FC_ERR_INVALID_ARG before anything is queued.
+ * The same handle must not run two steps concurrently on different streams
+ * (they share the workspace); consecutive calls on one stream are fine.
+ */
+FC_API fc_status fc_step(fc_handle* h, void* stream, int batch, const void* x, const int32_t* q_pos,
+                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int total_q,
+                  int total_k, void* k_cache, void* v_cache, void* out, float* importance,
+                  int accumulate);
+
+/*
+ * fc_topk_tracked — reselect the tracked positions of every sequence.
+ *   total_k       S (host int): length of `importance`, <= max_total_k.
+ *   importance    dev, float [S] as written by fc_step.
+ *   cu_seqlens_k  dev, int32 [B+1] (as for fc_step); a sequence whose range
+ *                 leaves [0, S) sets FC_DEVERR_CAND and gets a row of -1.
+ *   cand_lo/hi    dev, int32 [B]: sequence b's candidates are the positions
+ *                 cand_lo[b] <= j < cand_hi[b] (0 <= lo <= hi <= L_b), normally
+ *                 its decoded positions.
+ *   k_per_seq     dev, int32 [B] or NULL: number kept for sequence b
+ *                 (0 <= k_b <= k); NULL keeps k for every sequence.
+ *   k             row width of `tracked`, 0 <= k <= max_topk.
+ *   tracked       dev, int32 [B, k]: row b lists the kept positions ordered by
+ *                 importance descending, equal scores by position ascending;
+ *                 entries past min(k_b, number of candidates) are -1.
+ * Exact and deterministic: the same inputs give the same output bits.
+ */
+FC_API fc_status fc_topk_tracked(fc_handle* h, void* stream, int batch, int total_k,
+                          const float* importance,
+                          const int32_t* cu_seqlens_k, const int32_t* cand_lo,
+                          const int32_t* cand_hi, const int32_t* k_per_seq, int k,
+                          int32_t* tracked);
+
+/*
+ * fc_get_error — wait for the stream of the handle's last call, copy the
+ * device error word to *device_error_word (host) and clear it.
+ * Returns FC_OK when the word was 0, FC_ERR_TIMEOUT when it holds
+ * FC_DEVERR_TIMEOUT, otherwise FC_ERR_DEVICE_CHECK; FC_ERR_CUDA if the wait
+ * or the copy failed.
+ */
+FC_API fc_status fc_get_error(fc_handle* h, int32_t* device_error_word);
+
+/* Number of kernels the last fc_step / fc_topk_tracked call enqueued (host). */
+FC_API int fc_last_launch_count(const fc_handle* h);
+
+/*
+ * Per-kernel timing for measurement tools.  fc_profile(h, 1) makes every later
+ * fc_step / fc_topk_tracked record a CUDA event pair on its stream around each
+ * kernel it launches (up to 4096 launches); fc_profile(h, 0) stops recording.
+ * fc_profile_read waits for the recorded work, writes for each kernel slot
+ * (0 prep, 1 qkv_rope_scatter, 2 attention, 3 importance_finalize, 4 topk) the
+ * summed milliseconds to ms[slot] and the launch count to launches[slot]
+ * (host arrays of FC_PROFILE_SLOTS entries), and clears the record.
+ */
+#define FC_PROFILE_SLOTS 5
+FC_API fc_status fc_profile(fc_handle* h, int enable);
+FC_API fc_status fc_profile_read(fc_handle* h, float* ms, int* launches);
+
+/* Release the workspace and the handle (NULL is a no-op).  Waits for all work
+ * on the handle's device first (cudaDeviceSynchronize). */
+FC_API void fc_destroy(fc_handle* h);
+
+/* Static, human-readable name of a status. */
+FC_API const char* fc_status_str(fc_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLASHCACHE_H */

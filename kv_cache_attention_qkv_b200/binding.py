@@ -1,0 +1,217 @@
+"""ctypes binding of libflashcache.so (include/flashcache.h).
+
+Argument marshalling only: every step of the Flash-Cache path runs in the CUDA
+library.  Tensors are torch CUDA tensors; the binding checks dtype, device and
+contiguity (which the C ABI cannot see), passes raw pointers and the current
+torch stream, and turns a non-zero status into ``FlashCacheError``.  If the
+library is missing this module raises on import: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libflashcache.so")
+
+FC_DTYPE_BF16 = 0
+FC_DTYPE_FP32 = 1
+STATUS = {0: "FC_OK", -1: "FC_ERR_INVALID_ARG", -2: "FC_ERR_UNSUPPORTED", -3: "FC_ERR_CUDA",
+          -4: "FC_ERR_OOM", -5: "FC_ERR_DEVICE_CHECK", -6: "FC_ERR_TIMEOUT"}
+DEVERR = {0x01: "POS_RANGE", 0x02: "POS_DUP", 0x04: "SEQLENS", 0x08: "CAND", 0x10: "TIMEOUT"}
+EXPORTED = ("fc_create", "fc_step", "fc_topk_tracked", "fc_get_error", "fc_last_launch_count",
+            "fc_profile", "fc_profile_read", "fc_destroy", "fc_status_str")
+PROFILE_SLOTS = ("prep", "qkv_rope_scatter", "attention", "importance_finalize", "topk")
+
+
+class FlashCacheError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+class FcConfig(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("n_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("rope_theta", ctypes.c_double), ("dtype", ctypes.c_int),
+                ("max_batch", ctypes.c_int), ("max_total_q", ctypes.c_int),
+                ("max_total_k", ctypes.c_int), ("max_seqlen_q", ctypes.c_int),
+                ("max_pos", ctypes.c_int), ("max_topk", ctypes.c_int)]
+
+
+_lib = None
+
+
+def load_library(path: Optional[str] = None):
+    """Load libflashcache.so once and declare its signatures."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise FlashCacheError(-3, f"{p} is not built (run python -m kv_cache_attention_qkv_b200.build)")
+    lib = ctypes.CDLL(p)
+    vp, i32p, c_int = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.c_int
+    lib.fc_create.argtypes = [ctypes.POINTER(FcConfig), vp, ctypes.POINTER(vp)]
+    lib.fc_create.restype = c_int
+    lib.fc_step.argtypes = [vp, vp, c_int, vp, vp, vp, vp, c_int, c_int, vp, vp, vp, vp, c_int]
+    lib.fc_step.restype = c_int
+    lib.fc_topk_tracked.argtypes = [vp, vp, c_int, c_int, vp, vp, vp, vp, vp, c_int, vp]
+    lib.fc_topk_tracked.restype = c_int
+    lib.fc_get_error.argtypes = [vp, i32p]
+    lib.fc_get_error.restype = c_int
+    lib.fc_last_launch_count.argtypes = [vp]
+    lib.fc_last_launch_count.restype = c_int
+    lib.fc_profile.argtypes = [vp, c_int]
+    lib.fc_profile.restype = c_int
+    lib.fc_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(c_int)]
+    lib.fc_profile_read.restype = c_int
+    lib.fc_destroy.argtypes = [vp]
+    lib.fc_destroy.restype = None
+    lib.fc_status_str.argtypes = [c_int]
+    lib.fc_status_str.restype = ctypes.c_char_p
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class FlashCache:
+    """One Flash-Cache layer: W_qkv bound at construction, steps on demand."""
+
+    def __init__(self, w_qkv: torch.Tensor, *, hidden: int, n_heads: int, head_dim: int,
+                 rope_theta: float, max_batch: int, max_total_q: int, max_total_k: int,
+                 max_seqlen_q: int, max_pos: int, max_topk: int):
+        self.lib = load_library()
+        if w_qkv.dtype == torch.bfloat16:
+            self.dtype, dt = torch.bfloat16, FC_DTYPE_BF16
+        elif w_qkv.dtype == torch.float32:
+            self.dtype, dt = torch.float32, FC_DTYPE_FP32
+        else:
+            raise FlashCacheError(-1, f"w_qkv dtype {w_qkv.dtype} is neither bfloat16 nor float32")
+        if not (w_qkv.is_cuda and w_qkv.is_contiguous()):
+            raise FlashCacheError(-1, "w_qkv must be a contiguous CUDA tensor")
+        if tuple(w_qkv.shape) != (3 * n_heads * head_dim, hidden):
+            raise FlashCacheError(-1, f"w_qkv shape {tuple(w_qkv.shape)} != [3*H*d, hidden]")
+        self.w_qkv = w_qkv  # the library keeps the pointer: keep the tensor alive
+        self.hidden, self.n_heads, self.head_dim = hidden, n_heads, head_dim
+        self.cfg = FcConfig(hidden, n_heads, head_dim, float(rope_theta), dt, max_batch,
+                            max_total_q, max_total_k, max_seqlen_q, max_pos, max_topk)
+        self.device = w_qkv.device
+        h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            st = self.lib.fc_create(ctypes.byref(self.cfg), _ptr(w_qkv), ctypes.byref(h))
+        if st != 0:
+            raise FlashCacheError(st, "fc_create")
+        self._h = h
+
+    # ------------------------------------------------------------------ checks
+    def _check(self, t: torch.Tensor, name: str, dtype, ndim: Optional[int] = None):
+        if t.dtype != dtype or not t.is_cuda or t.device != self.device or not t.is_contiguous():
+            raise FlashCacheError(-1, f"{name}: need a contiguous {dtype} tensor on {self.device}")
+        if ndim is not None and t.dim() != ndim:
+            raise FlashCacheError(-1, f"{name}: need {ndim} dimensions, got {t.dim()}")
+
+    def step(self, x, q_pos, cu_seqlens_q, cu_seqlens_k, k_cache, v_cache, out,
+             importance=None, accumulate: bool = False, stream=None) -> None:
+        """Enqueue fc_step on ``stream`` (default: torch's current stream)."""
+        H, d = self.n_heads, self.head_dim
+        self._check(x, "x", self.dtype, 2)
+        self._check(q_pos, "q_pos", torch.int32, 1)
+        self._check(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+        self._check(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
+        for n, t in (("k_cache", k_cache), ("v_cache", v_cache), ("out", out)):
+            self._check(t, n, self.dtype, 3)
+            if t.shape[1:] != (H, d):
+                raise FlashCacheError(-1, f"{n}: trailing shape {tuple(t.shape[1:])} != ({H}, {d})")
+        T, S = x.shape[0], k_cache.shape[0]
+        B = cu_seqlens_q.shape[0] - 1
+        if (x.shape[1] != self.hidden or q_pos.shape[0] != T or out.shape[0] != T
+                or v_cache.shape[0] != S or cu_seqlens_k.shape[0] != B + 1):
+            raise FlashCacheError(-1, "fc_step: inconsistent shapes")
+        if importance is not None:
+            self._check(importance, "importance", torch.float32, 1)
+            if importance.shape[0] != S:
+                raise FlashCacheError(-1, "importance must have one entry per cache row")
+        st = self.lib.fc_step(self._h, _stream_handle(stream), B, _ptr(x), _ptr(q_pos),
+                              _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), T, S, _ptr(k_cache),
+                              _ptr(v_cache), _ptr(out), _ptr(importance), int(bool(accumulate)))
+        if st != 0:
+            raise FlashCacheError(st, "fc_step")
+
+    def topk_tracked(self, importance, cu_seqlens_k, cand_lo, cand_hi, k: int, tracked,
+                     k_per_seq=None, stream=None) -> None:
+        """Enqueue fc_topk_tracked; ``tracked`` is int32 [B, k]."""
+        self._check(importance, "importance", torch.float32, 1)
+        for n, t in (("cu_seqlens_k", cu_seqlens_k), ("cand_lo", cand_lo), ("cand_hi", cand_hi)):
+            self._check(t, n, torch.int32, 1)
+        B = cu_seqlens_k.shape[0] - 1
+        if k_per_seq is not None:
+            self._check(k_per_seq, "k_per_seq", torch.int32, 1)
+        self._check(tracked, "tracked", torch.int32, 2)
+        if tuple(tracked.shape) != (B, k) or cand_lo.shape[0] != B or cand_hi.shape[0] != B:
+            raise FlashCacheError(-1, "fc_topk_tracked: inconsistent shapes")
+        st = self.lib.fc_topk_tracked(self._h, _stream_handle(stream), B, importance.shape[0],
+                                      _ptr(importance), _ptr(cu_seqlens_k), _ptr(cand_lo),
+                                      _ptr(cand_hi), _ptr(k_per_seq), int(k), _ptr(tracked))
+        if st != 0:
+            raise FlashCacheError(st, "fc_topk_tracked")
+
+    def get_error(self) -> int:
+        """Wait for the last stream used and return (and clear) the device error word."""
+        w = ctypes.c_int32(0)
+        st = self.lib.fc_get_error(self._h, ctypes.byref(w))
+        if st not in (0, -5, -6):
+            raise FlashCacheError(st, "fc_get_error")
+        return int(w.value)
+
+    def profile(self, enable: bool) -> None:
+        """Record a CUDA event pair around every later kernel launch (or stop)."""
+        st = self.lib.fc_profile(self._h, int(bool(enable)))
+        if st != 0:
+            raise FlashCacheError(st, "fc_profile")
+
+    def profile_read(self):
+        """{kernel: (summed ms, launches)} since the last read; waits for the work."""
+        ms = (ctypes.c_float * len(PROFILE_SLOTS))()
+        n = (ctypes.c_int * len(PROFILE_SLOTS))()
+        st = self.lib.fc_profile_read(self._h, ms, n)
+        if st != 0:
+            raise FlashCacheError(st, "fc_profile_read")
+        return {name: (float(ms[i]), int(n[i])) for i, name in enumerate(PROFILE_SLOTS)}
+
+    @property
+    def last_launch_count(self) -> int:
+        return int(self.lib.fc_last_launch_count(self._h))
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            self.lib.fc_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+
+def describe_error_word(word: int):
+    return [name for bit, name in DEVERR.items() if word & bit]

@@ -1,0 +1,96 @@
+// Internal declarations shared by the host runtime and the kernels of
+// libflashcache.so.  Not part of the public ABI (include/flashcache.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/flashcache.h"
+
+namespace fc {
+
+// Query rows per attention work item of the tensor-core path and of the SIMT
+// path.  A work item is one (sequence, head, query tile).
+constexpr int kTcQTile = 128;
+constexpr int kSimtQTile = 16;
+
+// Importance is accumulated in fixed point (int64, 2^-40 units) so that the
+// sum over heads and query tiles is exact and independent of the order in
+// which work items finish.  One column sum is at most kSimtQTile..128 and a
+// key receives at most H * n_b contributions, far inside 2^23.
+constexpr double kImpScale = 1099511627776.0;  // 2^40
+constexpr double kImpInvScale = 1.0 / 1099511627776.0;
+
+// Work-list item: sequence, query tile, head.
+struct WorkItem {
+  int32_t seq;
+  int32_t tile_head;  // (qtile << 8) | head
+};
+
+struct Workspace {
+  void* q_buf = nullptr;                  // [max_total_q, H, d] dtype; rotated, pre-scaled q
+  int32_t* row_dst = nullptr;             // [max_total_q] cache row of query row, or -1
+  unsigned long long* imp_acc = nullptr;  // [max_total_k] fixed-point importance
+  WorkItem* items = nullptr;              // attention work list
+  int32_t* sched = nullptr;               // [0] = item count, [1] = dynamic item counter
+  int32_t* err = nullptr;                 // device error word
+  float* rope_cos = nullptr;              // [max_pos, d/2]
+  float* rope_sin = nullptr;              // [max_pos, d/2]
+  int max_items = 0;
+};
+
+// Shapes of one step, as the kernels see them.
+struct StepShape {
+  int B, T, S, D, H, d;
+  int max_pos, max_seqlen_q;
+};
+
+}  // namespace fc
+
+struct fc_handle {
+  fc_config cfg;
+  int device = 0;
+  int num_sms = 0;
+  bool tc_path = false;  // bf16 + d == 128 + D % 64 == 0 + (H*d) % 256 == 0
+  const void* w_qkv = nullptr;
+  fc::Workspace ws;
+  cudaStream_t last_stream = nullptr;
+  int last_launches = 0;
+  // optional per-kernel event timing (fc_profile)
+  bool profiling = false;
+  int prof_n = 0;
+  int prof_slot[4096];
+  cudaEvent_t* prof_ev = nullptr;  // 2 * 4096 events, created on first fc_profile(1)
+  CUtensorMap tm_w;  // W_qkv, bf16 tensor-core path
+  CUtensorMap tm_q;  // Q buffer, bf16 tensor-core path
+};
+
+namespace fc {
+
+// ---- launchers (each returns the CUDA error of its launch) -----------------
+cudaError_t launch_prep(const fc_handle* h, cudaStream_t st, const StepShape& s,
+                        const int32_t* q_pos, const int32_t* cu_q, const int32_t* cu_k,
+                        int qtile);
+cudaError_t launch_qkv_simt(const fc_handle* h, cudaStream_t st, const StepShape& s,
+                            const void* x, const int32_t* q_pos, void* k_cache, void* v_cache);
+cudaError_t launch_attn_simt(const fc_handle* h, cudaStream_t st, const StepShape& s,
+                             const int32_t* cu_q, const int32_t* cu_k, const void* k_cache,
+                             const void* v_cache, void* out, bool want_importance);
+cudaError_t launch_qkv_tc(const fc_handle* h, cudaStream_t st, const StepShape& s,
+                          const CUtensorMap& tm_x, const int32_t* q_pos, void* k_cache,
+                          void* v_cache);
+cudaError_t launch_attn_tc(const fc_handle* h, cudaStream_t st, const StepShape& s,
+                           const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                           const int32_t* cu_q, const int32_t* cu_k, void* out,
+                           bool want_importance);
+cudaError_t launch_importance_finalize(const fc_handle* h, cudaStream_t st, int S,
+                                       float* importance, int accumulate);
+cudaError_t launch_topk(const fc_handle* h, cudaStream_t st, int B, int S, const float* importance,
+                        const int32_t* cu_k, const int32_t* cand_lo, const int32_t* cand_hi,
+                        const int32_t* k_per_seq, int k, int32_t* tracked);
+
+// Dynamic shared memory the prep kernel needs for a given max_pos.
+size_t prep_smem_bytes(int max_pos, int max_batch);
+
+}  // namespace fc

@@ -1,0 +1,180 @@
+// Step preparation: validate the packed layout on the device, map every query
+// row to its cache row, and build the attention work list.
+//
+// The cache row of query row r of sequence b is cu_seqlens_k[b] + q_pos[r]
+// (Flash-Cache writes the refreshed K/V at the rows' absolute positions:
+// infernews post "Flash-dLLM: IO-aware KV caching and parallel decoding",
+// Flash-Cache paragraph).  Rows whose position is outside the sequence, or
+// shared with another row of the same sequence, get -1 and are never written.
+#include "fc_internal.h"
+
+namespace fc {
+namespace {
+
+__device__ __forceinline__ void set_err(int32_t* err, int bits) { atomicOr(err, bits); }
+
+// Sanity of sequence b's ranges; the same test is applied by every kernel
+// that trusts cu_seqlens, so that a bad sequence is skipped consistently.
+__device__ __forceinline__ bool seq_ok(const int32_t* cu_q, const int32_t* cu_k, int b, int B,
+                                       int T, int S, int max_pos, int max_n) {
+  int q0 = cu_q[b], q1 = cu_q[b + 1], k0 = cu_k[b], k1 = cu_k[b + 1];
+  bool ok = q0 >= 0 && q0 <= q1 && q1 <= T && k0 >= 0 && k0 <= k1 && k1 <= S &&
+            (k1 - k0) <= max_pos && (q1 - q0) <= max_n;
+  if (b == 0) ok = ok && q0 == 0 && k0 == 0;
+  if (b == B - 1) ok = ok && q1 == T && k1 == S;
+  return ok;
+}
+
+// Blocks 0..B-1: one sequence each.  Block B: the work list.
+__global__ void __launch_bounds__(512) prep_kernel(StepShape s, const int32_t* __restrict__ q_pos,
+                                                   const int32_t* __restrict__ cu_q,
+                                                   const int32_t* __restrict__ cu_k,
+                                                   int32_t* __restrict__ row_dst,
+                                                   WorkItem* __restrict__ items, int max_items,
+                                                   int32_t* __restrict__ sched,
+                                                   int32_t* __restrict__ err, int qtile) {
+  extern __shared__ uint32_t smem[];
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x, nt = blockDim.x;
+
+  if (b < s.B) {
+    const bool ok = seq_ok(cu_q, cu_k, b, s.B, s.T, s.S, s.max_pos, s.max_seqlen_q);
+    int q0 = min(max(cu_q[b], 0), s.T), q1 = min(max(cu_q[b + 1], q0), s.T);
+    if (!ok) {
+      if (tid == 0) set_err(err, FC_DEVERR_SEQLENS);
+      for (int r = q0 + tid; r < q1; r += nt) row_dst[r] = -1;
+      return;
+    }
+    const int k0 = cu_k[b], L = cu_k[b + 1] - k0;
+    const int words = (L + 31) >> 5;
+    uint32_t* seen = smem;
+    uint32_t* dup = smem + words;
+    for (int i = tid; i < 2 * words; i += nt) smem[i] = 0u;
+    __syncthreads();
+    bool bad_range = false;
+    for (int r = q0 + tid; r < q1; r += nt) {
+      int p = q_pos[r];
+      if (p < 0 || p >= L) {
+        bad_range = true;
+        continue;
+      }
+      uint32_t bit = 1u << (p & 31);
+      if (atomicOr(&seen[p >> 5], bit) & bit) atomicOr(&dup[p >> 5], bit);
+    }
+    if (bad_range) set_err(err, FC_DEVERR_POS_RANGE);
+    __syncthreads();
+    bool any_dup = false;
+    for (int r = q0 + tid; r < q1; r += nt) {
+      int p = q_pos[r];
+      int dst = -1;
+      if (p >= 0 && p < L) {
+        if (dup[p >> 5] & (1u << (p & 31)))
+          any_dup = true;
+        else
+          dst = k0 + p;
+      }
+      row_dst[r] = dst;
+    }
+    if (any_dup) set_err(err, FC_DEVERR_POS_DUP);
+    return;
+  }
+
+  // ---- work list: sequences by cache length descending (longest first), then
+  // for each sequence its items ordered (head, query tile) so that the tiles
+  // of one (sequence, head) that read the same K/V run close together.
+  int n2 = 1;
+  while (n2 < s.B) n2 <<= 1;
+  unsigned long long* key = reinterpret_cast<unsigned long long*>(smem);
+  int* cnt = reinterpret_cast<int*>(key + n2);  // [n2] items per sorted sequence, then offsets
+  for (int i = tid; i < n2; i += nt) {
+    unsigned long long k = 0ull;
+    if (i < s.B) {
+      bool ok = seq_ok(cu_q, cu_k, i, s.B, s.T, s.S, s.max_pos, s.max_seqlen_q);
+      int n = ok ? cu_q[i + 1] - cu_q[i] : 0;
+      int L = ok ? cu_k[i + 1] - cu_k[i] : 0;
+      // valid sequences with rows sort before everything else, then by L desc, b asc
+      unsigned long long live = (n > 0) ? 1ull : 0ull;
+      k = (live << 63) | ((unsigned long long)(unsigned)L << 32) |
+          (unsigned long long)(0xFFFFFFFFu - (unsigned)i);
+    }
+    key[i] = k;
+  }
+  __syncthreads();
+  // bitonic sort, descending
+  for (int size = 2; size <= n2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < n2; i += nt) {
+        int j = i ^ stride;
+        if (j > i) {
+          bool desc = ((i & size) == 0);
+          unsigned long long a = key[i], c = key[j];
+          if (desc ? (a < c) : (a > c)) {
+            key[i] = c;
+            key[j] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = tid; i < n2; i += nt) {
+    int c = 0;
+    if (i < s.B && (key[i] >> 63)) {
+      int bq = (int)(0xFFFFFFFFu - (unsigned)(key[i] & 0xFFFFFFFFull));
+      int n = cu_q[bq + 1] - cu_q[bq];
+      c = s.H * ((n + qtile - 1) / qtile);
+    }
+    cnt[i] = c;
+  }
+  __syncthreads();
+  if (tid == 0) {  // serial exclusive scan; B <= 4096
+    int run = 0;
+    for (int i = 0; i < s.B; ++i) {
+      int c = cnt[i];
+      cnt[i] = run;
+      run += c;
+    }
+    int total = min(run, max_items);
+    sched[0] = total;
+    sched[1] = 0;
+  }
+  __syncthreads();
+  for (int i = 0; i < s.B; ++i) {
+    if (!(key[i] >> 63)) break;
+    int bq = (int)(0xFFFFFFFFu - (unsigned)(key[i] & 0xFFFFFFFFull));
+    int n = cu_q[bq + 1] - cu_q[bq];
+    int nqt = (n + qtile - 1) / qtile;
+    int c = s.H * nqt;
+    int off = cnt[i];
+    for (int t = tid; t < c; t += nt) {
+      int hh = t / nqt, qt = t - hh * nqt;
+      if (off + t < max_items) items[off + t] = WorkItem{bq, (qt << 8) | hh};
+    }
+  }
+}
+
+}  // namespace
+
+size_t prep_smem_bytes(int max_pos, int max_batch) {
+  size_t bitmap = 2u * (size_t)((max_pos + 31) / 32) * sizeof(uint32_t);
+  int n2 = 1;
+  while (n2 < max_batch) n2 <<= 1;
+  size_t sortb = (size_t)n2 * (sizeof(unsigned long long) + sizeof(int));
+  return bitmap > sortb ? bitmap : sortb;
+}
+
+cudaError_t launch_prep(const fc_handle* h, cudaStream_t st, const StepShape& s,
+                        const int32_t* q_pos, const int32_t* cu_q, const int32_t* cu_k,
+                        int qtile) {
+  size_t smem = prep_smem_bytes(h->cfg.max_pos, h->cfg.max_batch);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  prep_kernel<<<s.B + 1, 512, smem, st>>>(s, q_pos, cu_q, cu_k, h->ws.row_dst, h->ws.items,
+                                           h->ws.max_items, h->ws.sched, h->ws.err, qtile);
+  return cudaGetLastError();
+}
+
+}  // namespace fc

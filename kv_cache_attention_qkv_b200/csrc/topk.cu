@@ -1,0 +1,194 @@
+// Importance finalisation and tracked-set reselection.
+//
+// Flash-Cache keeps tracking the top-k decoded tokens ranked by attention
+// importance (Flash-dLLM paper-digest page, Fig. 2 caption; infernews post
+// "Flash-dLLM: IO-aware KV caching and parallel decoding", Flash-Cache
+// paragraph: only newly decoded tokens and a few key positions chosen by
+// attention importance are refreshed).
+//
+// topk_tracked: one CTA per sequence.  An exact radix select (four 8-bit
+// digits of an order-preserving 32-bit key) finds the k-th largest score; all
+// larger scores are kept, equal ones in position order until k are kept, and
+// the kept set is sorted by (score desc, position asc).  The result does not
+// depend on thread timing.
+#include "fc_internal.h"
+
+namespace fc {
+namespace {
+
+__global__ void importance_finalize(int S, unsigned long long* __restrict__ acc,
+                                    float* __restrict__ imp, int accumulate) {
+  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < S; j += gridDim.x * blockDim.x) {
+    const double v = (double)(long long)acc[j] * kImpInvScale;
+    const float f = (float)v;
+    imp[j] = accumulate ? imp[j] + f : f;
+    acc[j] = 0ull;
+  }
+}
+
+// Order-preserving map float -> uint32 (larger float, larger key).
+__device__ __forceinline__ uint32_t fkey(float f) {
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+constexpr int TK_THREADS = 512;
+constexpr int TK_MAXK = 1024;
+
+__global__ void __launch_bounds__(TK_THREADS) topk_kernel(
+    int B, const float* __restrict__ imp, const int32_t* __restrict__ cu_k,
+    const int32_t* __restrict__ cand_lo, const int32_t* __restrict__ cand_hi,
+    const int32_t* __restrict__ k_per_seq, int k, int32_t* __restrict__ tracked,
+    int32_t* __restrict__ err, int S, int max_pos) {
+  __shared__ uint32_t hist[256];
+  __shared__ unsigned long long sel[TK_MAXK];
+  __shared__ int sh_digit, sh_remaining, sh_nsel, sh_run;
+  __shared__ int warp_cnt[TK_THREADS / 32];
+
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int32_t* row = tracked + (size_t)b * k;
+
+  const int k0 = cu_k[b], k1 = cu_k[b + 1];
+  const int lo = cand_lo[b], hi = cand_hi[b];
+  const int kb = k_per_seq ? k_per_seq[b] : k;
+  const int L = k1 - k0;
+  const bool ok = k0 >= 0 && k0 <= k1 && k1 <= S && L <= max_pos && lo >= 0 && lo <= hi &&
+                  hi <= L && kb >= 0 && kb <= k;
+  if (!ok) {
+    if (tid == 0) atomicOr(err, FC_DEVERR_CAND);
+    for (int i = tid; i < k; i += TK_THREADS) row[i] = -1;
+    return;
+  }
+  const int n = hi - lo;
+  const int want = min(kb, n);
+  const float* sc = imp + k0 + lo;
+
+  // ---- radix select of the want-th largest key
+  uint32_t prefix = 0u, mask = 0u;
+  int remaining = want;  // how many still to take at or below the current prefix
+  if (want > 0) {
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += TK_THREADS) hist[i] = 0u;
+      __syncthreads();
+      for (int i = tid; i < n; i += TK_THREADS) {
+        const uint32_t key = fkey(sc[i]);
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane l scans digits 255-8l .. 248-8l (descending)
+        uint32_t c[8], tot = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          c[t] = hist[255 - 8 * lane - t];
+          tot += c[t];
+        }
+        uint32_t incl = tot;
+        for (int o = 1; o < 32; o <<= 1) {
+          uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const uint32_t excl = incl - tot;
+        if ((int)excl < remaining && remaining <= (int)incl) {
+          uint32_t run = excl;
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            if ((int)run < remaining && remaining <= (int)(run + c[t])) {
+              sh_digit = 255 - 8 * lane - t;
+              sh_remaining = remaining - (int)run;
+            }
+            run += c[t];
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= (uint32_t)sh_digit << shift;
+      mask |= 0xFFu << shift;
+      remaining = sh_remaining;
+      __syncthreads();
+    }
+  }
+  const uint32_t thr = prefix;  // key of the want-th largest score
+  // `remaining` equal-to-thr candidates are kept, lowest positions first.
+
+  if (tid == 0) {
+    sh_nsel = 0;
+    sh_run = 0;
+  }
+  __syncthreads();
+  if (want > 0) {
+    for (int base = 0; base < n; base += TK_THREADS) {
+      const int i = base + tid;
+      uint32_t key = 0u;
+      bool gt = false, eq = false;
+      if (i < n) {
+        key = fkey(sc[i]);
+        gt = key > thr;
+        eq = key == thr;
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, eq);
+      if (lane == 0) warp_cnt[warp] = __popc(bal);
+      __syncthreads();
+      int before = sh_run;
+      for (int w = 0; w < warp; ++w) before += warp_cnt[w];
+      before += __popc(bal & ((1u << lane) - 1u));
+      const bool take = gt || (eq && before < remaining);
+      if (take) {
+        const int slot = atomicAdd(&sh_nsel, 1);
+        if (slot < TK_MAXK)
+          sel[slot] = ((unsigned long long)key << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)(lo + i));
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int tot = 0;
+        for (int w = 0; w < TK_THREADS / 32; ++w) tot += warp_cnt[w];
+        sh_run += tot;
+      }
+      __syncthreads();
+    }
+  }
+  // ---- sort the kept set: key desc, position asc (composite descending)
+  int m2 = 1;
+  while (m2 < want) m2 <<= 1;
+  for (int i = want + tid; i < m2; i += TK_THREADS) sel[i] = 0ull;
+  __syncthreads();
+  for (int size = 2; size <= m2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < m2; i += TK_THREADS) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool desc = (i & size) == 0;
+          const unsigned long long a = sel[i], c = sel[j];
+          if (desc ? (a < c) : (a > c)) {
+            sel[i] = c;
+            sel[j] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = tid; i < k; i += TK_THREADS)
+    row[i] = i < want ? (int32_t)(0xFFFFFFFFu - (uint32_t)(sel[i] & 0xFFFFFFFFull)) : -1;
+}
+
+}  // namespace
+
+cudaError_t launch_importance_finalize(const fc_handle* h, cudaStream_t st, int S,
+                                       float* importance, int accumulate) {
+  if (S <= 0) return cudaSuccess;
+  int blocks = (S + 255) / 256;
+  if (blocks > h->num_sms * 8) blocks = h->num_sms * 8;
+  importance_finalize<<<blocks, 256, 0, st>>>(S, h->ws.imp_acc, importance, accumulate);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const fc_handle* h, cudaStream_t st, int B, int S, const float* importance,
+                        const int32_t* cu_k, const int32_t* cand_lo, const int32_t* cand_hi,
+                        const int32_t* k_per_seq, int k, int32_t* tracked) {
+  topk_kernel<<<B, TK_THREADS, 0, st>>>(B, importance, cu_k, cand_lo, cand_hi, k_per_seq, k,
+                                        tracked, h->ws.err, S, h->cfg.max_pos);
+  return cudaGetLastError();
+}
+
+}  // namespace fc

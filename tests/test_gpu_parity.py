@@ -1,0 +1,195 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_attention_qkv_b200 import workloads
+import fc_testlib as tl
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu(cuda_ok):
+    return cuda_ok
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "small_varlen", "layer_b1"])
+def test_full_parity(name):
+    """Every output element of small workloads against the oracle."""
+    inp = workloads.generate(name)
+    gpu = tl.run_gpu(inp)
+    assert gpu["err"] == 0
+    ref = tl.run_oracle(inp)
+    tl.compare_step(inp, gpu, ref, range(inp.batch))
+    tl.assert_unwritten_rows_unchanged(inp, gpu)
+    # importance of every key of the batch, not only the sampled sequences
+    tl.assert_close(gpu["importance"], ref["importance"], tl.TOL[inp.dtype], "importance")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,seqs", [("batch32_uniform", [0, 13, 31]),
+                                       ("batch32_varlen", [0, 5, 17, 30])])
+def test_full_size_sampled_parity(name, seqs):
+    """Full-size workloads, same launch configuration as the bench; the oracle
+    recomputes sampled sequences (sequences are independent)."""
+    inp = workloads.generate(name)
+    gpu = tl.run_gpu(inp)
+    assert gpu["err"] == 0
+    ref = tl.run_oracle(inp, seqs=seqs)
+    tl.compare_step(inp, gpu, ref, seqs)
+    tl.assert_unwritten_rows_unchanged(inp, gpu)
+    # properties that hold for every sequence at any size
+    imp = gpu["importance"]
+    for b in range(inp.batch):
+        n = inp.cu_seqlens_q[b + 1] - inp.cu_seqlens_q[b]
+        tot = imp[inp.seq_slice_k(b)].sum()
+        assert abs(tot - inp.n_heads * n) <= 1e-3 * inp.n_heads * n, (b, tot)
+    assert np.isfinite(gpu["out"]).all()
+
+
+def test_topk_kernel_is_exact_on_gpu_importance():
+    """fc_topk_tracked on the GPU's own importance equals the oracle's
+    reselection of those same fp32 values, bit for bit."""
+    inp = workloads.generate("small_varlen")
+    gpu = tl.run_gpu(inp)
+    ref_tr = oracle.topk_tracked(gpu["importance"], inp.cu_seqlens_k, inp.cand_lo, inp.cand_hi,
+                                 inp.topk, int(inp.topk.max()))
+    np.testing.assert_array_equal(gpu["tracked"], ref_tr)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_topk_ties_and_ragged_candidates(seed):
+    """Planted ties, empty candidate ranges, k above the candidate count."""
+    rng = np.random.default_rng(seed)
+    B = 7
+    L = rng.integers(1, 3000, B)
+    L[2] = 1
+    cu = np.zeros(B + 1, np.int32)
+    cu[1:] = np.cumsum(L)
+    imp = (rng.integers(0, 50, cu[-1]) * 0.125).astype(np.float32)
+    imp[cu[3]:cu[4]] = 1.0  # one sequence made entirely of ties
+    lo = np.array([rng.integers(0, l + 1) for l in L], np.int32)
+    hi = np.array([rng.integers(a, l + 1) for a, l in zip(lo, L)], np.int32)
+    lo[5], hi[5] = 3, 3  # empty
+    K = 300
+    kb = rng.integers(0, K + 1, B).astype(np.int32)
+    inp = workloads.generate("tiny_fp32")
+    dev = tl.upload(inp)
+    layer = tl.make_layer(inp, dev["w"], max_topk=K, max_total_k=int(cu[-1]), max_pos=int(L.max()),
+                          max_batch=B)
+    t = lambda a: torch.from_numpy(a).cuda()
+    tracked = torch.full((B, K), -7, dtype=torch.int32, device="cuda")
+    layer.topk_tracked(t(imp), t(cu), t(lo), t(hi), K, tracked, k_per_seq=t(kb))
+    assert layer.get_error() == 0
+    ref = oracle.topk_tracked(imp.astype(np.float64), cu, lo, hi, kb, K)
+    np.testing.assert_array_equal(tracked.cpu().numpy(), ref)
+
+
+def test_rerun_is_bit_identical():
+    """The step is deterministic: a second run from the same inputs gives the
+    same bytes (importance is summed in order-independent fixed point)."""
+    inp = workloads.generate("small_varlen")
+    a = tl.run_gpu(inp)
+    b = tl.run_gpu(inp)
+    assert np.array_equal(a["out"], b["out"])
+    assert np.array_equal(a["importance"], b["importance"])
+    assert np.array_equal(a["tracked"], b["tracked"])
+    assert torch.equal(a["dev"]["k_cache"], b["dev"]["k_cache"])
+
+
+def test_step_is_idempotent_in_place():
+    """Running the same step twice on the same cache leaves it as after one."""
+    inp = workloads.generate("small_varlen")
+    dev = tl.upload(inp)
+    layer = tl.make_layer(inp, dev["w"])
+    a = tl.run_gpu(inp, layer=layer, dev=dev)
+    k1 = dev["k_cache"].clone()
+    b = tl.run_gpu(inp, layer=layer, dev=dev)
+    assert torch.equal(k1, dev["k_cache"])
+    assert np.array_equal(a["out"], b["out"])
+
+
+def test_accumulate_adds_importance():
+    inp = workloads.generate("small_varlen")
+    dev = tl.upload(inp)
+    layer = tl.make_layer(inp, dev["w"])
+    T, H, d = inp.total_q, inp.n_heads, inp.head_dim
+    out = torch.empty((T, H, d), device="cuda", dtype=torch.bfloat16)
+    imp = torch.zeros(inp.total_k, device="cuda")
+    layer.step(dev["x"], dev["q_pos"], dev["cu_q"], dev["cu_k"], dev["k_cache"], dev["v_cache"], out, imp)
+    one = imp.clone()
+    layer.step(dev["x"], dev["q_pos"], dev["cu_q"], dev["cu_k"], dev["k_cache"], dev["v_cache"], out, imp,
+               accumulate=True)
+    torch.cuda.synchronize()
+    assert torch.equal(imp, one + one)
+
+
+def test_without_importance_and_empty_query():
+    inp = workloads.generate("small_varlen")
+    gpu = tl.run_gpu(inp, want_importance=False)
+    ref = tl.run_oracle(inp)
+    tl.assert_close(gpu["out"], ref["out"], 1e-2, "out without importance")
+    # T = 0: nothing written, importance zeroed
+    layer, dev = gpu["layer"], gpu["dev"]
+    B = inp.batch
+    cu0 = torch.zeros(B + 1, dtype=torch.int32, device="cuda")
+    imp = torch.full((inp.total_k,), 5.0, device="cuda")
+    before = dev["k_cache"].clone()
+    layer.step(dev["x"][:0], dev["q_pos"][:0], cu0, dev["cu_k"], dev["k_cache"], dev["v_cache"],
+               torch.empty((0, inp.n_heads, inp.head_dim), device="cuda", dtype=torch.bfloat16), imp)
+    torch.cuda.synchronize()
+    assert torch.equal(before, dev["k_cache"]) and float(imp.abs().max()) == 0.0
+    assert layer.get_error() == 0
+
+
+def test_single_key_sequence_returns_value():
+    """L_b = 1 with a single query row at position 0: attention returns v."""
+    inp = workloads.generate("small_varlen", batch=1)
+    # shrink to one row attending a one-row cache
+    inp.q_pos = np.array([0], np.int32)
+    inp.x = inp.x[:1]
+    inp.cu_seqlens_q = np.array([0, 1], np.int32)
+    inp.cu_seqlens_k = np.array([0, 1], np.int32)
+    inp.k_cache, inp.v_cache = inp.k_cache[:1], inp.v_cache[:1]
+    inp.cand_lo, inp.cand_hi, inp.topk = (np.array([0], np.int32), np.array([1], np.int32),
+                                          np.array([1], np.int32))
+    gpu = tl.run_gpu(inp)
+    ref = tl.run_oracle(inp)
+    tl.compare_step(inp, gpu, ref, [0])
+    tl.assert_close(gpu["out"][0], ref["v_cache"][0], 1e-2, "o = v")
+    assert abs(gpu["importance"][0] - inp.n_heads) < 1e-3
+
+
+@pytest.mark.parametrize("bad", ["range", "dup", "seqlens", "cand"])
+def test_device_checks_set_error_word(bad):
+    from kv_cache_attention_qkv_b200.binding import describe_error_word
+
+    inp = workloads.generate("small_varlen")
+    if bad == "range":
+        inp.q_pos = inp.q_pos.copy()
+        inp.q_pos[3] = 10_000
+    elif bad == "dup":
+        inp.q_pos = inp.q_pos.copy()
+        inp.q_pos[5] = inp.q_pos[4]
+    elif bad == "seqlens":
+        inp.cu_seqlens_q = inp.cu_seqlens_q.copy()
+        inp.cu_seqlens_q[1] = inp.cu_seqlens_q[2] + 1  # not monotone
+    else:
+        inp.cand_hi = inp.cand_hi.copy()
+        inp.cand_hi[0] = 10 ** 6
+    prior_k = inp.k_cache.copy()
+    gpu = tl.run_gpu(inp)
+    names = describe_error_word(gpu["err"])
+    expect = {"range": "POS_RANGE", "dup": "POS_DUP", "seqlens": "SEQLENS", "cand": "CAND"}[bad]
+    assert expect in names, names
+    # the offending rows were not written anywhere
+    if bad in ("range", "dup"):
+        k_now = gpu["dev"]["k_cache"].float().cpu().numpy()
+        S = inp.total_k
+        assert k_now.shape[0] == S
+        if bad == "dup":
+            row = inp.seq_slice_k(0).start + inp.q_pos[4]
+            np.testing.assert_array_equal(k_now[row], prior_k[row])
+    assert tl.run_gpu(workloads.generate("small_varlen"), layer=gpu["layer"])["err"] == 0
