@@ -149,9 +149,12 @@ fc_status fc_create(const fc_config* cfg, const void* w_qkv, fc_handle** out) {
   h->num_sms = nsm;
   h->w_qkv = w_qkv;
   const int H = cfg->n_heads, d = cfg->head_dim, half = d / 2;
-  h->tc_path = false;
+  const bool tc_shape = cfg->dtype == FC_DTYPE_BF16 && d == 128 && cfg->hidden % 64 == 0 &&
+                        (H % 2) == 0;
+  h->tc_gemm = tc_shape;
+  h->tc_attn = false;
 
-  const int qtile = h->tc_path ? fc::kTcQTile : fc::kSimtQTile;
+  const int qtile = h->tc_attn ? fc::kTcQTile : fc::kSimtQTile;
   h->ws.max_items = H * (cfg->max_total_q / qtile + cfg->max_batch + 1);
 
   fc::Workspace& w = h->ws;
@@ -191,12 +194,12 @@ fc_status fc_create(const fc_config* cfg, const void* w_qkv, fc_handle** out) {
        cudaMemset(w.err, 0, sizeof(int32_t)) == cudaSuccess &&
        cudaMemset(w.sched, 0, 4 * sizeof(int32_t)) == cudaSuccess &&
        cudaMemset(w.row_dst, 0xFF, (size_t)cfg->max_total_q * sizeof(int32_t)) == cudaSuccess;
-  if (ok && h->tc_path) {
+  if (ok && h->tc_gemm)
     ok = fc::encode_bf16_2d(&h->tm_w, w_qkv, (uint64_t)3 * H * d, (uint64_t)cfg->hidden,
-                            (uint64_t)cfg->hidden * 2, 256, 64) &&
-         fc::encode_bf16_2d(&h->tm_q, w.q_buf, (uint64_t)cfg->max_total_q * H, (uint64_t)d,
+                            (uint64_t)cfg->hidden * 2, 256, 64);
+  if (ok && h->tc_attn)
+    ok = fc::encode_bf16_2d(&h->tm_q, w.q_buf, (uint64_t)cfg->max_total_q * H, (uint64_t)d,
                             (uint64_t)d * 2, 128, 64);
-  }
   if (!ok || cudaDeviceSynchronize() != cudaSuccess) {
     cudaGetLastError();
     free_workspace(h);
@@ -240,11 +243,18 @@ fc_status fc_step(fc_handle* h, void* stream, int batch, const void* x, const in
   {
     ProfScope ps(h, st, 0);
     e = fc::launch_prep(h, st, s, q_pos, cu_seqlens_q, cu_seqlens_k,
-                        h->tc_path ? fc::kTcQTile : fc::kSimtQTile);
+                        h->tc_attn ? fc::kTcQTile : fc::kSimtQTile);
   }
   if (e != cudaSuccess) return FC_ERR_CUDA;
   h->last_launches++;
-  {
+  if (h->tc_gemm) {
+    CUtensorMap tm_x;
+    if (!fc::encode_bf16_2d(&tm_x, x, (uint64_t)total_q, (uint64_t)c.hidden,
+                            (uint64_t)c.hidden * 2, 128, 64))
+      return FC_ERR_CUDA;
+    ProfScope ps(h, st, 1);
+    e = fc::launch_qkv_tc(h, st, s, tm_x, q_pos, k_cache, v_cache);
+  } else {
     ProfScope ps(h, st, 1);
     e = fc::launch_qkv_simt(h, st, s, x, q_pos, k_cache, v_cache);
   }

@@ -52,7 +52,9 @@ struct fc_handle {
   fc_config cfg;
   int device = 0;
   int num_sms = 0;
-  bool tc_path = false;  // bf16 + d == 128 + D % 64 == 0 + (H*d) % 256 == 0
+  // tensor-core kernels: bf16, head_dim 128, hidden % 64 == 0, H even
+  bool tc_gemm = false;
+  bool tc_attn = false;
   const void* w_qkv = nullptr;
   fc::Workspace ws;
   cudaStream_t last_stream = nullptr;
@@ -89,6 +91,10 @@ cudaError_t launch_importance_finalize(const fc_handle* h, cudaStream_t st, int 
 cudaError_t launch_topk(const fc_handle* h, cudaStream_t st, int B, int S, const float* importance,
                         const int32_t* cu_k, const int32_t* cand_lo, const int32_t* cand_hi,
                         const int32_t* k_per_seq, int k, int32_t* tracked);
+
+size_t qkv_tc_smem_bytes();
+bool encode_bf16_2d(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols,
+                    uint64_t row_stride_bytes, uint32_t box_rows, uint32_t box_cols);
 
 // Dynamic shared memory the prep kernel needs for a given max_pos.
 size_t prep_smem_bytes(int max_pos, int max_batch);

@@ -15,6 +15,8 @@ Five workloads are defined, named by what they are:
                      window 16 or 64 and tracking budget 48/64/80 per sequence.
 * ``small_varlen``   a few-second ragged case for element-wise parity: B=3,
                      hidden 256, 4 heads x 128, caches of 129..700 rows.
+* ``small_d64``      bf16 with head_dim 64 (the CUDA-core path): B=2, hidden
+                     96, 3 heads x 64, caches of 200 and 333 rows.
 
 The shapes follow LLaDA-8B (the model the Flash-dLLM pages evaluate); weights
 and caches are random, there is no dataset and no checkpoint.
@@ -30,7 +32,8 @@ from typing import Dict, List, Optional
 
 import numpy as np
 
-WORKLOADS = ("tiny_fp32", "layer_b1", "batch32_uniform", "batch32_varlen", "small_varlen")
+WORKLOADS = ("tiny_fp32", "layer_b1", "batch32_uniform", "batch32_varlen", "small_varlen",
+             "small_d64")
 
 
 @dataclasses.dataclass
@@ -157,6 +160,13 @@ def generate(name: str, seed: Optional[int] = None, batch: Optional[int] = None)
             first = -(-lo // w) * w
             last = L - w
             starts.append(int(first + w * rng.integers(0, (last - first) // w + 1)))
+    elif name == "small_d64":
+        dtype, D, H, d, theta, w_std = "bf16", 96, 3, 64, 1.0e4, 0.1
+        B = batch or 2
+        lens = [[200, 333][i % 2] for i in range(B)]
+        windows = [[16, 64][i % 2] for i in range(B)]
+        budgets = [[40, 64][i % 2] for i in range(B)]
+        starts = [[48, 256][i % 2] for i in range(B)]
     else:  # small_varlen
         dtype, D, H, d, theta, w_std = "bf16", 256, 4, 128, 5.0e5, 0.0625
         B = batch or 3
@@ -205,5 +215,7 @@ def describe(name: str) -> Dict[str, object]:
                                cache="U[600,2048]", query="48/64/80 tracked + 16/64 window"),
         "small_varlen": dict(dtype="bf16", B=3, hidden=256, heads=4, head_dim=128,
                              cache="700,129,333", query="80+64, 48+16, 100+64"),
+        "small_d64": dict(dtype="bf16", B=2, hidden=96, heads=3, head_dim=64,
+                          cache="200,333", query="40+16, 64+64"),
     }
     return table[name]

@@ -15,7 +15,7 @@ def _need_gpu(cuda_ok):
     return cuda_ok
 
 
-@pytest.mark.parametrize("name", ["tiny_fp32", "small_varlen", "layer_b1"])
+@pytest.mark.parametrize("name", ["tiny_fp32", "small_d64", "small_varlen", "layer_b1"])
 def test_full_parity(name):
     """Every output element of small workloads against the oracle."""
     inp = workloads.generate(name)
