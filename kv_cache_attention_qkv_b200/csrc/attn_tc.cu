@@ -1,0 +1,511 @@
+// Bidirectional variable-length attention over the whole per-sequence KV
+// cache on the tensor cores, with the per-key column sums of the attention
+// probabilities ("attention importance") as a side output.
+//
+// Flash-dLLM (paper-digest page, Fig. 2 caption): the fixed-size query of a
+// sequence attends bidirectionally to its full KV cache; the tracked positions
+// are reselected by attention importance.  Queries of different lengths share
+// one launch through block scheduling (infernews post "Flash-dLLM: IO-aware KV
+// caching and parallel decoding", Flash-Cache paragraph).
+//
+// One work item = (sequence b, head h, 128-row query tile).  The importance
+// needs the final softmax normalisation of every row before columns are
+// summed, so the cache is scanned twice:
+//   pass 1: S = Q K^T per 128-key tile, online row max m and sum l;
+//   pass 2: S = Q K^T again, P = 2^(S - m - log2 l) (final probabilities),
+//           O += P V, colsum(P) = ones * P, both on the tensor cores.
+// Q arrives pre-scaled by log2(e)/sqrt(d) from the projection epilogue, so
+// scores are already in the exp2 domain.
+//
+// Roles (one CTA per SM, persistent over the work list):
+//   warp 0     TMA producer: Q tile, then K tiles (pass 1), then K and V tiles
+//              (pass 2) into a ring of four 32 KiB slots;
+//   warp 1     TMEM allocation and tcgen05.mma issue: S into two TMEM buffers,
+//              O and the column sums into their own TMEM columns;
+//   warps 2-5  softmax: one query row per thread; writes P (bf16, 128-byte
+//              swizzle) to shared memory, adds the column sums to the
+//              fixed-point importance accumulator, writes O.
+#include <cuda_bf16.h>
+
+#include "fc_internal.h"
+#include "ptx.cuh"
+
+namespace fc {
+namespace {
+
+constexpr int QT = 128, KT = 128, HD = 128;
+constexpr int SLOTS = 4;
+constexpr uint32_t HALF_BYTES = 128 * 128;       // 128 rows x 64 bf16
+constexpr uint32_t TILE_BYTES = 2 * HALF_BYTES;  // 128 rows x 128 bf16
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_SLOT = TILE_BYTES;
+constexpr uint32_t OFF_P = OFF_SLOT + SLOTS * TILE_BYTES;
+constexpr uint32_t OFF_ONES = OFF_P + TILE_BYTES;
+constexpr uint32_t ONES_BYTES = 2048;
+constexpr uint32_t OFF_BARS = OFF_ONES + ONES_BYTES;
+constexpr int THREADS = 192;
+// TMEM columns
+constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_CS = 384;
+
+constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(128, 128, 0, 0);   // Q K^T, both K-major
+constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, 128, 0, 1);  // P V, V MN-major
+constexpr uint32_t IDESC_CS = ptx::idesc_bf16_f32(128, 128, 0, 1);  // ones P, P MN-major
+
+struct AttnParams {
+  int H, max_T;
+  const WorkItem* items;
+  const int32_t* sched;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  __nv_bfloat16* out;
+  unsigned long long* imp_acc;
+  int want_imp;
+  int32_t* err;
+};
+
+struct __align__(8) AttnBars {
+  unsigned long long qfull, qfree;
+  unsigned long long full[SLOTS], empty[SLOTS];
+  unsigned long long sfull[2], sfree[2];
+  unsigned long long pready, pfree;
+  unsigned long long ofull, ofree;
+  unsigned long long drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct Item {
+  int b, qt, h, q0, nrows, k0, L, ntiles;
+};
+
+__device__ __forceinline__ Item load_item(const AttnParams& p, int it) {
+  const WorkItem w = p.items[it];
+  Item r;
+  r.b = w.seq;
+  r.qt = w.tile_head >> 8;
+  r.h = w.tile_head & 0xFF;
+  r.q0 = p.cu_q[r.b];
+  const int n = p.cu_q[r.b + 1] - r.q0;
+  r.nrows = min(QT, n - r.qt * QT);
+  r.k0 = p.cu_k[r.b];
+  r.L = p.cu_k[r.b + 1] - r.k0;
+  r.ntiles = (r.L + KT - 1) / KT;
+  return r;
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, int x, int y,
+                                            int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = ptx::smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  AttnBars* bars = reinterpret_cast<AttnBars*>(smem + OFF_BARS);
+  volatile int* abort_flag = &bars->abort_flag;
+  auto bar = [](unsigned long long& b) { return ptx::smem_u32(&b); };
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_items = p.sched[0];
+
+  // constant all-ones operand (8 rows x 128 columns, two 64-column atoms)
+  for (int i = tid; i < (int)(ONES_BYTES / 4); i += THREADS)
+    reinterpret_cast<uint32_t*>(smem + OFF_ONES)[i] = 0x3F803F80u;
+  fence_proxy_async_smem();
+  if (tid == 0) {
+    ptx::mbar_init(bar(bars->qfull), 1);
+    ptx::mbar_init(bar(bars->qfree), 1);
+    for (int s = 0; s < SLOTS; ++s) {
+      ptx::mbar_init(bar(bars->full[s]), 1);
+      ptx::mbar_init(bar(bars->empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(bar(bars->sfull[s]), 1);
+      ptx::mbar_init(bar(bars->sfree[s]), 4);
+    }
+    ptx::mbar_init(bar(bars->pready), 4);
+    ptx::mbar_init(bar(bars->pfree), 1);
+    ptx::mbar_init(bar(bars->ofull), 1);
+    ptx::mbar_init(bar(bars->ofree), 4);
+    ptx::mbar_init(bar(bars->drain), 1);
+    bars->abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tm_q);
+    ptx::prefetch_tmap(&tm_k);
+    ptx::prefetch_tmap(&tm_v);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(&bars->tmem_base), 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  bool failed = false;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- producer
+      uint32_t prod = 0;  // slot production counter
+      int issued_phase[SLOTS];
+      for (int s = 0; s < SLOTS; ++s) issued_phase[s] = -1;
+      int q_issued_phase = -1;
+      uint32_t ic = 0;
+      auto load_tile = [&](const CUtensorMap* tm, int h, int row) -> bool {
+        const uint32_t s = prod % SLOTS, ph = (prod / SLOTS) & 1u;
+        if (!ptx::mbar_wait(bar(bars->empty[s]), ph ^ 1u, abort_flag)) return false;
+        const uint32_t dst = base + OFF_SLOT + s * TILE_BYTES;
+        ptx::mbar_arrive_expect_tx(bar(bars->full[s]), TILE_BYTES);
+        tma_load_3d(dst, tm, 0, h, row, bar(bars->full[s]));
+        tma_load_3d(dst + HALF_BYTES, tm, 64, h, row, bar(bars->full[s]));
+        issued_phase[s] = (int)ph;
+        ++prod;
+        return true;
+      };
+      for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
+        const Item t = load_item(p, it);
+        if (!ptx::mbar_wait(bar(bars->qfree), (ic & 1u) ^ 1u, abort_flag)) {
+          failed = true;
+          break;
+        }
+        ptx::mbar_arrive_expect_tx(bar(bars->qfull), TILE_BYTES);
+        const int qrow = t.h * p.max_T + t.q0 + t.qt * QT;
+        ptx::tma_load_2d(base + OFF_Q, &tm_q, 0, qrow, bar(bars->qfull));
+        ptx::tma_load_2d(base + OFF_Q + HALF_BYTES, &tm_q, 64, qrow, bar(bars->qfull));
+        q_issued_phase = (int)(ic & 1u);
+        for (int j = 0; j < t.ntiles && !failed; ++j)
+          if (!load_tile(&tm_k, t.h, t.k0 + j * KT)) failed = true;
+        for (int j = 0; j < t.ntiles && !failed; ++j) {
+          if (!load_tile(&tm_k, t.h, t.k0 + j * KT) || !load_tile(&tm_v, t.h, t.k0 + j * KT))
+            failed = true;
+        }
+      }
+      if (failed) {
+        *abort_flag = 1;
+        const unsigned long long t0 = ptx::globaltimer();
+        for (int s = 0; s < SLOTS; ++s)
+          if (issued_phase[s] >= 0)
+            while (!ptx::mbar_try_wait(bar(bars->full[s]), (uint32_t)issued_phase[s]) &&
+                   ptx::globaltimer() - t0 < ptx::kWaitLimitNs) {
+            }
+        if (q_issued_phase >= 0)
+          while (!ptx::mbar_try_wait(bar(bars->qfull), (uint32_t)q_issued_phase) &&
+                 ptx::globaltimer() - t0 < ptx::kWaitLimitNs) {
+          }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      uint32_t cons = 0;  // slot consumption index base (production order)
+      uint32_t scnt = 0;  // S tiles issued
+      uint32_t pcnt = 0;  // pready completions consumed
+      uint32_t ic = 0;
+      const uint32_t q_addr = base + OFF_Q;
+      const uint32_t p_addr = base + OFF_P;
+      const uint32_t ones_addr = base + OFF_ONES;
+      auto slot_wait = [&](uint32_t idx) -> bool {
+        return ptx::mbar_wait(bar(bars->full[idx % SLOTS]), (idx / SLOTS) & 1u, abort_flag);
+      };
+      auto slot_addr = [&](uint32_t idx) { return base + OFF_SLOT + (idx % SLOTS) * TILE_BYTES; };
+      // S[sb] = Q K^T for the K tile in production slot idx
+      auto issue_s = [&](uint32_t idx) -> bool {
+        const uint32_t sb = scnt & 1u;
+        if (!ptx::mbar_wait(bar(bars->sfree[sb]), ((scnt >> 1) & 1u) ^ 1u, abort_flag)) return false;
+        if (!slot_wait(idx)) return false;
+        ptx::tc_fence_after();
+        const uint32_t k_addr = slot_addr(idx);
+#pragma unroll
+        for (int k = 0; k < HD / 16; ++k) {
+          const uint32_t off = (uint32_t)(k >> 2) * HALF_BYTES + (uint32_t)(k & 3) * 32;
+          ptx::mma_bf16_ss(tmem + TM_S0 + sb * 128, ptx::smem_desc(q_addr + off, 16, 1024),
+                           ptx::smem_desc(k_addr + off, 16, 1024), IDESC_S, k > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(bar(bars->sfull[sb]));
+        ptx::mma_commit(bar(bars->empty[idx % SLOTS]));
+        ++scnt;
+        return true;
+      };
+      // O += P V and CS = ones P for the V tile in production slot idx
+      auto issue_pv = [&](uint32_t idx, bool first) -> bool {
+        if (!ptx::mbar_wait(bar(bars->pready), pcnt & 1u, abort_flag)) return false;
+        ++pcnt;
+        if (!slot_wait(idx)) return false;
+        ptx::tc_fence_after();
+        const uint32_t v_addr = slot_addr(idx);
+#pragma unroll
+        for (int k = 0; k < KT / 16; ++k) {
+          // A = P (K-major over keys); B = V (MN-major: d contiguous, keys are K)
+          const uint32_t poff = (uint32_t)(k >> 2) * HALF_BYTES + (uint32_t)(k & 3) * 32;
+          ptx::mma_bf16_ss(tmem + TM_O, ptx::smem_desc(p_addr + poff, 16, 1024),
+                           ptx::smem_desc(v_addr + (uint32_t)k * 2048, HALF_BYTES, 1024), IDESC_PV,
+                           (first && k == 0) ? 0u : 1u);
+        }
+        if (p.want_imp) {
+#pragma unroll
+          for (int k = 0; k < QT / 16; ++k) {
+            // A = ones (rows alias one 8-row atom: SBO = 0); B = P^T (MN-major:
+            // keys contiguous, query rows are K)
+            const uint32_t aoff = (uint32_t)(k >> 2) * 1024 + (uint32_t)(k & 3) * 32;
+            ptx::mma_bf16_ss(tmem + TM_CS, ptx::smem_desc(ones_addr + aoff, 16, 0),
+                             ptx::smem_desc(p_addr + (uint32_t)k * 2048, HALF_BYTES, 1024),
+                             IDESC_CS, k > 0 ? 1u : 0u);
+          }
+        }
+        ptx::mma_commit(bar(bars->empty[idx % SLOTS]));
+        ptx::mma_commit(bar(bars->pfree));
+        return true;
+      };
+      for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
+        const Item t = load_item(p, it);
+        if (!ptx::mbar_wait(bar(bars->qfull), ic & 1u, abort_flag)) {
+          failed = true;
+          break;
+        }
+        // pass 1: S tiles only
+        for (int j = 0; j < t.ntiles && !failed; ++j)
+          if (!issue_s(cons + (uint32_t)j)) failed = true;
+        if (failed) break;
+        const uint32_t base2 = cons + (uint32_t)t.ntiles;
+        // the previous item's O must have been read out before P V overwrites it
+        if (!ptx::mbar_wait(bar(bars->ofree), (ic & 1u) ^ 1u, abort_flag)) {
+          failed = true;
+          break;
+        }
+        for (int j = 0; j < t.ntiles && !failed; ++j) {
+          if (!issue_s(base2 + 2u * (uint32_t)j)) {
+            failed = true;
+            break;
+          }
+          if (j == t.ntiles - 1) ptx::mma_commit(bar(bars->qfree));
+          if (j > 0 && !issue_pv(base2 + 2u * (uint32_t)(j - 1) + 1u, j == 1)) failed = true;
+        }
+        if (failed) break;
+        if (!issue_pv(base2 + 2u * (uint32_t)(t.ntiles - 1) + 1u, t.ntiles == 1)) {
+          failed = true;
+          break;
+        }
+        ptx::mma_commit(bar(bars->ofull));
+        cons = base2 + 2u * (uint32_t)t.ntiles;
+      }
+      if (failed) {
+        *abort_flag = 1;
+        ptx::mma_commit(bar(bars->drain));
+        const unsigned long long t0 = ptx::globaltimer();
+        while (!ptx::mbar_try_wait(bar(bars->drain), 0u) &&
+               ptx::globaltimer() - t0 < ptx::kWaitLimitNs) {
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------- softmax warps
+    const int quad = warp & 3;
+    const int rl = quad * 32 + lane;  // query row inside the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t p_addr = base + OFF_P;
+    uint32_t scnt = 0, pfcnt = 0, ic = 0;
+
+    // Add the column sums of the previous P tile (tile index jt) to the
+    // fixed-point importance accumulator: every TMEM row of CS holds the same
+    // sums, so thread `lane` of quadrant `quad` takes column 32*quad + lane.
+    auto flush_colsum = [&](const Item& t, int jt) {
+      uint32_t r[32];
+      ptx::tmem_ld32(tmem + lane_off + TM_CS + (uint32_t)(quad * 32), r);
+      ptx::tmem_wait_ld();
+      float v = 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (e == lane) v = __uint_as_float(r[e]);
+      const int key = jt * KT + quad * 32 + lane;
+      if (key < t.L)
+        atomicAdd(&p.imp_acc[t.k0 + key], (unsigned long long)__double2ll_rn((double)v * kImpScale));
+    };
+    // Load S tile (128 fp32 columns of this thread's row) and release its buffer.
+    auto load_s = [&](uint32_t (&s)[128]) -> bool {
+      const uint32_t sb = scnt & 1u;
+      if (!ptx::mbar_wait(bar(bars->sfull[sb]), (scnt >> 1) & 1u, abort_flag)) return false;
+      ptx::tc_fence_after();
+      const uint32_t ta = tmem + lane_off + TM_S0 + sb * 128;
+      ptx::tmem_ld32(ta + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      ptx::tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      ptx::tmem_ld32(ta + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+      ptx::tmem_ld32(ta + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      ptx::tmem_wait_ld();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(bars->sfree[sb]));
+      ++scnt;
+      return true;
+    };
+
+    for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
+      const Item t = load_item(p, it);
+      const bool row_ok = rl < t.nrows;
+      uint32_t s[128];
+      // ---- pass 1: row max and normaliser
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < t.ntiles; ++j) {
+        if (!load_s(s)) {
+          failed = true;
+          break;
+        }
+        const int kmax = t.L - j * KT;  // keys >= kmax are outside the sequence
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c < kmax) tmax = fmaxf(tmax, __uint_as_float(s[c]));
+        const float mn = fmaxf(m, tmax);
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c < kmax) acc += ex2(__uint_as_float(s[c]) - mn);
+        l = l * ex2(m - mn) + acc;
+        m = mn;
+      }
+      if (failed) break;
+      const float lse = m + __log2f(l);
+      // ---- pass 2: final probabilities -> P (smem), column sums, O
+      for (int j = 0; j < t.ntiles; ++j) {
+        if (!load_s(s)) {
+          failed = true;
+          break;
+        }
+        const int kmax = row_ok ? t.L - j * KT : 0;
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const float p0 = c < kmax ? ex2(__uint_as_float(s[c]) - lse) : 0.f;
+          const float p1 = c + 1 < kmax ? ex2(__uint_as_float(s[c + 1]) - lse) : 0.f;
+          pk[c / 2] = pack_bf16(p0, p1);
+        }
+        if (j > 0) {
+          // P buffer free (previous P V and colsum done): read that colsum
+          if (!ptx::mbar_wait(bar(bars->pfree), pfcnt & 1u, abort_flag)) {
+            failed = true;
+            break;
+          }
+          ++pfcnt;
+          ptx::tc_fence_after();
+          if (p.want_imp) flush_colsum(t, j - 1);
+        }
+        // P row rl: keys 0..63 in half 0, 64..127 in half 1; 16-byte chunk
+        // index XOR (row & 7) is the 128-byte swizzle.
+#pragma unroll
+        for (int ch = 0; ch < 16; ++ch) {
+          const uint32_t half = (uint32_t)(ch >> 3);
+          const uint32_t c16 = (uint32_t)(ch & 7) ^ (uint32_t)(rl & 7);
+          const uint32_t addr = p_addr + half * HALF_BYTES + (uint32_t)rl * 128 + (c16 << 4);
+          st_shared_v4(addr, pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        }
+        fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(bars->pready));
+      }
+      if (failed) break;
+      if (!ptx::mbar_wait(bar(bars->pfree), pfcnt & 1u, abort_flag)) {
+        failed = true;
+        break;
+      }
+      ++pfcnt;
+      ptx::tc_fence_after();
+      if (p.want_imp) flush_colsum(t, t.ntiles - 1);
+      // ---- O (already normalised) -> out
+      if (!ptx::mbar_wait(bar(bars->ofull), ic & 1u, abort_flag)) {
+        failed = true;
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t ta = tmem + lane_off + TM_O;
+      ptx::tmem_ld32(ta + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      ptx::tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      ptx::tmem_ld32(ta + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+      ptx::tmem_ld32(ta + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      ptx::tmem_wait_ld();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(bars->ofree));
+      if (row_ok) {
+        uint4* dst = reinterpret_cast<uint4*>(
+            p.out + ((size_t)(t.q0 + t.qt * QT + rl) * p.H + t.h) * HD);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          uint4 w;
+          w.x = pack_bf16(__uint_as_float(s[8 * q + 0]), __uint_as_float(s[8 * q + 1]));
+          w.y = pack_bf16(__uint_as_float(s[8 * q + 2]), __uint_as_float(s[8 * q + 3]));
+          w.z = pack_bf16(__uint_as_float(s[8 * q + 4]), __uint_as_float(s[8 * q + 5]));
+          w.w = pack_bf16(__uint_as_float(s[8 * q + 6]), __uint_as_float(s[8 * q + 7]));
+          dst[q] = w;
+        }
+      }
+    }
+    if (failed) *abort_flag = 1;
+  }
+
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (tid == 0 && bars->abort_flag) atomicOr(p.err, FC_DEVERR_TIMEOUT);
+  if (warp == 1) ptx::tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+size_t attn_tc_smem_bytes() { return OFF_BARS + sizeof(AttnBars) + 1024; }
+
+cudaError_t launch_attn_tc(const fc_handle* h, cudaStream_t st, const StepShape& s,
+                           const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                           const int32_t* cu_q, const int32_t* cu_k, void* out,
+                           bool want_importance) {
+  AttnParams p;
+  p.H = s.H;
+  p.max_T = h->cfg.max_total_q;
+  p.items = h->ws.items;
+  p.sched = h->ws.sched;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.out = (__nv_bfloat16*)out;
+  p.imp_acc = h->ws.imp_acc;
+  p.want_imp = want_importance ? 1 : 0;
+  p.err = h->ws.err;
+  const size_t smem = attn_tc_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  attn_tc_kernel<<<h->num_sms, THREADS, smem, st>>>(h->tm_q, tm_k, tm_v, p);
+  return cudaGetLastError();
+}
+
+}  // namespace fc

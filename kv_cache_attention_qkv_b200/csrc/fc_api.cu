@@ -83,6 +83,22 @@ bool encode_bf16_2d(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t c
   return r == CUDA_SUCCESS;
 }
 
+// 3-D bf16 tensor map over a KV cache [S, H, 128]: box = 128 rows of one head,
+// 64 columns (one 128-byte swizzle row), so one (sequence, head) key tile is
+// two boxes.
+bool encode_kv_3d(CUtensorMap* tm, const void* cache, int S, int H) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)S};
+  cuuint64_t strides[2] = {256, (cuuint64_t)H * 256};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(cache), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace fc
 
 extern "C" {
@@ -152,7 +168,7 @@ fc_status fc_create(const fc_config* cfg, const void* w_qkv, fc_handle** out) {
   const bool tc_shape = cfg->dtype == FC_DTYPE_BF16 && d == 128 && cfg->hidden % 64 == 0 &&
                         (H % 2) == 0;
   h->tc_gemm = tc_shape;
-  h->tc_attn = false;
+  h->tc_attn = tc_shape;
 
   const int qtile = h->tc_attn ? fc::kTcQTile : fc::kSimtQTile;
   h->ws.max_items = H * (cfg->max_total_q / qtile + cfg->max_batch + 1);
@@ -199,7 +215,8 @@ fc_status fc_create(const fc_config* cfg, const void* w_qkv, fc_handle** out) {
                             (uint64_t)cfg->hidden * 2, 256, 64);
   if (ok && h->tc_attn)
     ok = fc::encode_bf16_2d(&h->tm_q, w.q_buf, (uint64_t)cfg->max_total_q * H, (uint64_t)d,
-                            (uint64_t)d * 2, 128, 64);
+                            (uint64_t)d * 2, 128, 64) &&
+         cudaMemset(w.q_buf, 0, (size_t)cfg->max_total_q * H * d * es) == cudaSuccess;
   if (!ok || cudaDeviceSynchronize() != cudaSuccess) {
     cudaGetLastError();
     free_workspace(h);
@@ -260,7 +277,14 @@ fc_status fc_step(fc_handle* h, void* stream, int batch, const void* x, const in
   }
   if (e != cudaSuccess) return FC_ERR_CUDA;
   h->last_launches++;
-  {
+  if (h->tc_attn) {
+    CUtensorMap tm_k, tm_v;
+    if (!fc::encode_kv_3d(&tm_k, k_cache, total_k, c.n_heads) ||
+        !fc::encode_kv_3d(&tm_v, v_cache, total_k, c.n_heads))
+      return FC_ERR_CUDA;
+    ProfScope ps(h, st, 2);
+    e = fc::launch_attn_tc(h, st, s, tm_k, tm_v, cu_seqlens_q, cu_seqlens_k, out, want_imp);
+  } else {
     ProfScope ps(h, st, 2);
     e = fc::launch_attn_simt(h, st, s, cu_seqlens_q, cu_seqlens_k, k_cache, v_cache, out,
                              want_imp);

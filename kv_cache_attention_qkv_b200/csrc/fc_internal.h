@@ -93,6 +93,8 @@ cudaError_t launch_topk(const fc_handle* h, cudaStream_t st, int B, int S, const
                         const int32_t* k_per_seq, int k, int32_t* tracked);
 
 size_t qkv_tc_smem_bytes();
+size_t attn_tc_smem_bytes();
+bool encode_kv_3d(CUtensorMap* tm, const void* cache, int S, int H);
 bool encode_bf16_2d(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols,
                     uint64_t row_stride_bytes, uint32_t box_rows, uint32_t box_cols);
 

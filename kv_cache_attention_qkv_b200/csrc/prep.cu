@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(512) prep_kernel(StepShape s, const int32_t* _
       int n = ok ? cu_q[i + 1] - cu_q[i] : 0;
       int L = ok ? cu_k[i + 1] - cu_k[i] : 0;
       // valid sequences with rows sort before everything else, then by L desc, b asc
-      unsigned long long live = (n > 0) ? 1ull : 0ull;
+      unsigned long long live = (n > 0 && L > 0) ? 1ull : 0ull;
       k = (live << 63) | ((unsigned long long)(unsigned)L << 32) |
           (unsigned long long)(0xFFFFFFFFu - (unsigned)i);
     }

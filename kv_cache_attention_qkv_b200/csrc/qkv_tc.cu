@@ -6,7 +6,8 @@
 // C[T, 3*H*128] = X[T, D] * W_qkv[3*H*128, D]^T is never written: each
 // 128 x 256 output tile (two heads) lives in TMEM, and the epilogue rotates q
 // and k by RoPE at the row's position and stores
-//   q * log2(e)/sqrt(d) -> Q buffer [T, H, d] (bf16),
+//   q * log2(e)/sqrt(d) -> Q buffer (bf16; [H, max_T, d] when the tensor-core
+//     attention reads it, else [T, H, d]),
 //   k, v (bf16, round to nearest even) -> cache row cu_seqlens_k[b] + q_pos[r].
 //
 // Structure (one CTA per SM, persistent over output tiles):
@@ -41,6 +42,7 @@ struct QkvParams {
   const float* rcos;
   const float* rsin;
   __nv_bfloat16* q_buf;
+  size_t q_rs, q_hs;  // element strides of a query row and of a head in the Q buffer
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
   float q_scale;
@@ -267,7 +269,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 lo[e] *= sc;
                 hi[e] *= sc;
               }
-              __nv_bfloat16* qrow = p.q_buf + ((size_t)row * p.H + hh) * HD;
+              __nv_bfloat16* qrow = p.q_buf + (size_t)row * p.q_rs + (size_t)hh * p.q_hs;
               store32(qrow + c, lo);
               store32(qrow + half + c, hi);
             }
@@ -313,6 +315,13 @@ cudaError_t launch_qkv_tc(const fc_handle* h, cudaStream_t st, const StepShape& 
   p.rcos = h->ws.rope_cos;
   p.rsin = h->ws.rope_sin;
   p.q_buf = (__nv_bfloat16*)h->ws.q_buf;
+  if (h->tc_attn) {  // [H, max_T, d]: one head's query rows contiguous for TMA
+    p.q_rs = HD;
+    p.q_hs = (size_t)h->cfg.max_total_q * HD;
+  } else {  // [T, H, d]
+    p.q_rs = (size_t)s.H * HD;
+    p.q_hs = HD;
+  }
   p.k_cache = (__nv_bfloat16*)k_cache;
   p.v_cache = (__nv_bfloat16*)v_cache;
   p.q_scale = (float)(1.4426950408889634 / sqrt((double)HD));
