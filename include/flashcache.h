@@ -191,6 +191,41 @@ FC_API int fc_last_launch_count(const fc_handle* h);
 FC_API fc_status fc_profile(fc_handle* h, int enable);
 FC_API fc_status fc_profile_read(fc_handle* h, float* ms, int* launches);
 
+/*
+ * fc_attention_noalloc — attention and importance without any device
+ * allocation.  The paper has no counterpart to this entry point: it exists for
+ * callers that cannot call cudaMalloc (a runtime or host application that owns
+ * all device memory, a plug-in running inside another process's context, a
+ * pool handed over to a caching allocator) and so cannot create a handle,
+ * whose workspace fc_create allocates.
+ *
+ * For query rows that are already projected and rotated, it computes what
+ * fc_step computes after its projection: out[r] = softmax(q_r K_b^T/sqrt(d)) V_b
+ * over every row of sequence b's cache, and importance[j] = sum over heads and
+ * query rows of the probability of key j (overwritten, no accumulate).
+ *   dtype          FC_DTYPE_BF16 or FC_DTYPE_FP32 (q, caches and out)
+ *   q              dev, [T, H, d]: rotated queries, not scaled
+ *   cu_seqlens_q/k dev, int32 [B+1], as for fc_step (sequences with ranges
+ *                  outside [0, T) / [0, S) are skipped)
+ *   k_cache, v_cache dev, [S, H, d], only read
+ *   out            dev, [T, H, d];  importance  dev, float [S]
+ * Limits: S <= FC_NOALLOC_MAX_KEYS, d <= 256, B and H <= 65535; larger sizes
+ * return FC_ERR_UNSUPPORTED before anything is queued.
+ * Its scratch (a fixed-point accumulator of FC_NOALLOC_MAX_KEYS + 32 int64,
+ * 512 KiB) is a static array in the library's device image: every GPU that
+ * loads the library holds it until the process exits, and every call shares
+ * it.  Each call clears the part it uses on `stream` first; calls whose work
+ * overlaps on the GPU (two streams, or two threads) race on it.  The first
+ * call on a device looks up the array's device address (once per device);
+ * make that first call before any stream capture.
+ */
+#define FC_NOALLOC_MAX_KEYS 65536
+FC_API fc_status fc_attention_noalloc(void* stream, int dtype, int batch, int n_heads,
+                                      int head_dim, const void* q, const int32_t* cu_seqlens_q,
+                                      const int32_t* cu_seqlens_k, int total_q, int total_k,
+                                      const void* k_cache, const void* v_cache, void* out,
+                                      float* importance);
+
 /* Release the workspace and the handle (NULL is a no-op).  Waits for all work
  * on the handle's device first (cudaDeviceSynchronize). */
 FC_API void fc_destroy(fc_handle* h);

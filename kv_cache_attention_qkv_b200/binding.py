@@ -23,7 +23,7 @@ STATUS = {0: "FC_OK", -1: "FC_ERR_INVALID_ARG", -2: "FC_ERR_UNSUPPORTED", -3: "F
           -4: "FC_ERR_OOM", -5: "FC_ERR_DEVICE_CHECK", -6: "FC_ERR_TIMEOUT"}
 DEVERR = {0x01: "POS_RANGE", 0x02: "POS_DUP", 0x04: "SEQLENS", 0x08: "CAND", 0x10: "TIMEOUT"}
 EXPORTED = ("fc_create", "fc_step", "fc_topk_tracked", "fc_get_error", "fc_last_launch_count",
-            "fc_profile", "fc_profile_read", "fc_destroy", "fc_status_str")
+            "fc_profile", "fc_profile_read", "fc_attention_noalloc", "fc_destroy", "fc_status_str")
 PROFILE_SLOTS = ("prep", "qkv_rope_scatter", "attention", "importance_finalize", "topk")
 
 
@@ -68,6 +68,9 @@ def load_library(path: Optional[str] = None):
     lib.fc_profile.restype = c_int
     lib.fc_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(c_int)]
     lib.fc_profile_read.restype = c_int
+    lib.fc_attention_noalloc.argtypes = [vp, c_int, c_int, c_int, c_int, vp, vp, vp, c_int, c_int,
+                                         vp, vp, vp, vp]
+    lib.fc_attention_noalloc.restype = c_int
     lib.fc_destroy.argtypes = [vp]
     lib.fc_destroy.restype = None
     lib.fc_status_str.argtypes = [c_int]
