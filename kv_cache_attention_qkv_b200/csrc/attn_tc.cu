@@ -11,20 +11,22 @@
 // One work item = (sequence b, head h, 128-row query tile).  The importance
 // needs the final softmax normalisation of every row before columns are
 // summed, so the cache is scanned twice:
-//   pass 1: S = Q K^T per 128-key tile, online row max m and sum l;
+//   pass 1: S = Q K^T per 128-key tile, row max m and sum l;
 //   pass 2: S = Q K^T again, P = 2^(S - m - log2 l) (final probabilities),
-//           O += P V, colsum(P) = ones * P, both on the tensor cores.
+//           O += P V and colsum(P) = ones * P, both on the tensor cores.
 // Q arrives pre-scaled by log2(e)/sqrt(d) from the projection epilogue, so
 // scores are already in the exp2 domain.
 //
 // Roles (one CTA per SM, persistent over the work list):
-//   warp 0     TMA producer: Q tile, then K tiles (pass 1), then K and V tiles
-//              (pass 2) into a ring of four 32 KiB slots;
-//   warp 1     TMEM allocation and tcgen05.mma issue: S into two TMEM buffers,
-//              O and the column sums into their own TMEM columns;
-//   warps 2-5  softmax: one query row per thread; writes P (bf16, 128-byte
-//              swizzle) to shared memory, adds the column sums to the
-//              fixed-point importance accumulator, writes O.
+//   warp 0      TMA producer: Q tile, then K tiles (pass 1), then K and V
+//               tiles (pass 2) into a ring of four 32 KiB slots;
+//   warp 1      TMEM allocation and tcgen05.mma issue: S into two TMEM
+//               buffers, O and the column sums into their own TMEM columns;
+//   warps 2-17  softmax: warp w owns TMEM lane quadrant w % 4 (32 query rows,
+//               one per thread) and a 32-column quarter (w - 2) / 4 of every
+//               128-column tile.  Four warps per scheduler keep the exp2
+//               pipe fed; the quarters' row statistics are merged once per
+//               item through shared memory.
 #include <cuda_bf16.h>
 
 #include "fc_internal.h"
@@ -35,6 +37,10 @@ namespace {
 
 constexpr int QT = 128, KT = 128, HD = 128;
 constexpr int SLOTS = 4;
+constexpr int SOFTMAX_WARPS = 16;
+constexpr int PARTS = 4;         // column quarters per row quadrant
+constexpr int CPW = KT / PARTS;  // columns per softmax warp
+constexpr int THREADS = 64 + 32 * SOFTMAX_WARPS;
 constexpr uint32_t HALF_BYTES = 128 * 128;       // 128 rows x 64 bf16
 constexpr uint32_t TILE_BYTES = 2 * HALF_BYTES;  // 128 rows x 128 bf16
 constexpr uint32_t OFF_Q = 0;
@@ -42,8 +48,9 @@ constexpr uint32_t OFF_SLOT = TILE_BYTES;
 constexpr uint32_t OFF_P = OFF_SLOT + SLOTS * TILE_BYTES;
 constexpr uint32_t OFF_ONES = OFF_P + TILE_BYTES;
 constexpr uint32_t ONES_BYTES = 2048;
-constexpr uint32_t OFF_BARS = OFF_ONES + ONES_BYTES;
-constexpr int THREADS = 192;
+constexpr uint32_t OFF_STAT = OFF_ONES + ONES_BYTES;
+constexpr uint32_t STAT_BYTES = 2 * PARTS * 2 * 128 * 4;  // [parity][part][m, l][row]
+constexpr uint32_t OFF_BARS = OFF_STAT + STAT_BYTES;
 // TMEM columns
 constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_CS = 384;
 
@@ -69,6 +76,7 @@ struct __align__(8) AttnBars {
   unsigned long long sfull[2], sfree[2];
   unsigned long long pready, pfree;
   unsigned long long ofull, ofree;
+  unsigned long long statbar;
   unsigned long long drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -124,6 +132,15 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, AttnParams p) {
@@ -151,12 +168,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(bar(bars->sfull[s]), 1);
-      ptx::mbar_init(bar(bars->sfree[s]), 4);
+      ptx::mbar_init(bar(bars->sfree[s]), SOFTMAX_WARPS);
     }
-    ptx::mbar_init(bar(bars->pready), 4);
+    ptx::mbar_init(bar(bars->pready), SOFTMAX_WARPS);
     ptx::mbar_init(bar(bars->pfree), 1);
     ptx::mbar_init(bar(bars->ofull), 1);
-    ptx::mbar_init(bar(bars->ofree), 4);
+    ptx::mbar_init(bar(bars->ofree), SOFTMAX_WARPS);
+    ptx::mbar_init(bar(bars->statbar), SOFTMAX_WARPS);
     ptx::mbar_init(bar(bars->drain), 1);
     bars->abort_flag = 0;
     ptx::fence_mbar_init();
@@ -331,36 +349,36 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // ---------------------------------------------------------- softmax warps
     const int quad = warp & 3;
+    const int part = (warp - 2) >> 2;
     const int rl = quad * 32 + lane;  // query row inside the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t p_addr = base + OFF_P;
+    const int col0 = CPW * part;      // first column of this warp in a tile
+    // this warp's 32 keys are 4 of the 8 16-byte chunks of one 64-key half of P
+    const uint32_t p_row = base + OFF_P + (uint32_t)(col0 >> 6) * HALF_BYTES + (uint32_t)rl * 128;
+    const uint32_t chunk0 = (uint32_t)((col0 & 63) >> 3);
+    float* stat = reinterpret_cast<float*>(smem + OFF_STAT);  // [parity][part][m, l][row]
     uint32_t scnt = 0, pfcnt = 0, ic = 0;
 
-    // Add the column sums of the previous P tile (tile index jt) to the
-    // fixed-point importance accumulator: every TMEM row of CS holds the same
-    // sums, so thread `lane` of quadrant `quad` takes column 32*quad + lane.
+    // Column sums of the previous P tile (tile jt): every TMEM row of CS holds
+    // the same sums; warp (quad, part) takes columns col0 + 8*quad .. +7.
     auto flush_colsum = [&](const Item& t, int jt) {
-      uint32_t r[32];
-      ptx::tmem_ld32(tmem + lane_off + TM_CS + (uint32_t)(quad * 32), r);
+      uint32_t r[8];
+      tmem_ld8(tmem + lane_off + TM_CS + (uint32_t)(col0 + 8 * quad), r);
       ptx::tmem_wait_ld();
       float v = 0.f;
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
+      for (int e = 0; e < 8; ++e)
         if (e == lane) v = __uint_as_float(r[e]);
-      const int key = jt * KT + quad * 32 + lane;
-      if (key < t.L)
+      const int key = jt * KT + col0 + 8 * quad + lane;
+      if (lane < 8 && key < t.L)
         atomicAdd(&p.imp_acc[t.k0 + key], (unsigned long long)__double2ll_rn((double)v * kImpScale));
     };
-    // Load S tile (128 fp32 columns of this thread's row) and release its buffer.
-    auto load_s = [&](uint32_t (&s)[128]) -> bool {
+    // This thread's 32 columns of the next S tile; the buffer is released at once.
+    auto load_s = [&](uint32_t (&sv)[32]) -> bool {
       const uint32_t sb = scnt & 1u;
       if (!ptx::mbar_wait(bar(bars->sfull[sb]), (scnt >> 1) & 1u, abort_flag)) return false;
       ptx::tc_fence_after();
-      const uint32_t ta = tmem + lane_off + TM_S0 + sb * 128;
-      ptx::tmem_ld32(ta + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-      ptx::tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-      ptx::tmem_ld32(ta + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-      ptx::tmem_ld32(ta + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      ptx::tmem_ld32(tmem + lane_off + TM_S0 + sb * 128 + (uint32_t)col0, sv);
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       __syncwarp();
@@ -371,43 +389,76 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
       const Item t = load_item(p, it);
-      const bool row_ok = rl < t.nrows;
-      uint32_t s[128];
-      // ---- pass 1: row max and normaliser
+      uint32_t sv[32];
+      // ---- pass 1: max and normaliser of this warp's 32-column quarter
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < t.ntiles; ++j) {
-        if (!load_s(s)) {
+        if (!load_s(sv)) {
           failed = true;
           break;
         }
-        const int kmax = t.L - j * KT;  // keys >= kmax are outside the sequence
-        float tmax = -INFINITY;
+        const int kmax = t.L - j * KT - col0;  // columns >= kmax are outside the sequence
+        if (kmax <= 0) continue;
+        float x[32];
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c < kmax) tmax = fmaxf(tmax, __uint_as_float(s[c]));
-        const float mn = fmaxf(m, tmax);
-        float acc = 0.f;
+        for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(sv[c]);
+        if (kmax < 32) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c < kmax) acc += ex2(__uint_as_float(s[c]) - mn);
-        l = l * ex2(m - mn) + acc;
+          for (int c = 0; c < 32; ++c)
+            if (c >= kmax) x[c] = -INFINITY;
+        }
+        float mx[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+        for (int c = 4; c < 32; ++c) mx[c & 3] = fmaxf(mx[c & 3], x[c]);
+        const float mn = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
+        float sm[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 32; ++c) sm[c & 3] += ex2(x[c] - mn);
+        l = l * ex2(m - mn) + ((sm[0] + sm[1]) + (sm[2] + sm[3]));
         m = mn;
       }
       if (failed) break;
-      const float lse = m + __log2f(l);
-      // ---- pass 2: final probabilities -> P (smem), column sums, O
+      // merge the four quarters of every row once per item
+      float* st_par = stat + (ic & 1u) * (PARTS * 256);
+      st_par[part * 256 + rl] = m;
+      st_par[part * 256 + 128 + rl] = l;
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(bars->statbar));
+      if (!ptx::mbar_wait(bar(bars->statbar), ic & 1u, abort_flag)) {
+        failed = true;
+        break;
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < PARTS; ++q) M = fmaxf(M, st_par[q * 256 + rl]);
+      float Ls = 0.f;
+#pragma unroll
+      for (int q = 0; q < PARTS; ++q) {
+        const float mq = st_par[q * 256 + rl];
+        if (mq != -INFINITY) Ls += st_par[q * 256 + 128 + rl] * ex2(mq - M);
+      }
+      // rows past the query tile's end get lse = +inf, i.e. P = 0
+      const float lse = rl < t.nrows ? M + __log2f(Ls) : INFINITY;
+      // ---- pass 2: final probabilities -> P (smem); P V and colsum on the MMA
       for (int j = 0; j < t.ntiles; ++j) {
-        if (!load_s(s)) {
+        if (!load_s(sv)) {
           failed = true;
           break;
         }
-        const int kmax = row_ok ? t.L - j * KT : 0;
-        uint32_t pk[64];
+        const int kmax = t.L - j * KT - col0;
+        uint32_t pk[16];
+        if (kmax >= 32) {
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float p0 = c < kmax ? ex2(__uint_as_float(s[c]) - lse) : 0.f;
-          const float p1 = c + 1 < kmax ? ex2(__uint_as_float(s[c + 1]) - lse) : 0.f;
-          pk[c / 2] = pack_bf16(p0, p1);
+          for (int c = 0; c < 32; c += 2)
+            pk[c / 2] = pack_bf16(ex2(__uint_as_float(sv[c]) - lse),
+                                  ex2(__uint_as_float(sv[c + 1]) - lse));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = c < kmax ? ex2(__uint_as_float(sv[c]) - lse) : 0.f;
+            const float p1 = c + 1 < kmax ? ex2(__uint_as_float(sv[c + 1]) - lse) : 0.f;
+            pk[c / 2] = pack_bf16(p0, p1);
+          }
         }
         if (j > 0) {
           // P buffer free (previous P V and colsum done): read that colsum
@@ -419,14 +470,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           ptx::tc_fence_after();
           if (p.want_imp) flush_colsum(t, j - 1);
         }
-        // P row rl: keys 0..63 in half 0, 64..127 in half 1; 16-byte chunk
-        // index XOR (row & 7) is the 128-byte swizzle.
+        // 16-byte chunk index XOR (row & 7) is the 128-byte swizzle
 #pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {
-          const uint32_t half = (uint32_t)(ch >> 3);
-          const uint32_t c16 = (uint32_t)(ch & 7) ^ (uint32_t)(rl & 7);
-          const uint32_t addr = p_addr + half * HALF_BYTES + (uint32_t)rl * 128 + (c16 << 4);
-          st_shared_v4(addr, pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        for (int ch = 0; ch < 4; ++ch) {
+          const uint32_t c16 = (chunk0 + (uint32_t)ch) ^ (uint32_t)(rl & 7);
+          st_shared_v4(p_row + (c16 << 4), pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2],
+                       pk[4 * ch + 3]);
         }
         fence_proxy_async_smem();
         ptx::tc_fence_before();
@@ -447,25 +496,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       }
       ptx::tc_fence_after();
-      const uint32_t ta = tmem + lane_off + TM_O;
-      ptx::tmem_ld32(ta + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-      ptx::tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-      ptx::tmem_ld32(ta + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-      ptx::tmem_ld32(ta + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      ptx::tmem_ld32(tmem + lane_off + TM_O + (uint32_t)col0, sv);
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(bars->ofree));
-      if (row_ok) {
+      if (rl < t.nrows) {
         uint4* dst = reinterpret_cast<uint4*>(
-            p.out + ((size_t)(t.q0 + t.qt * QT + rl) * p.H + t.h) * HD);
+            p.out + ((size_t)(t.q0 + t.qt * QT + rl) * p.H + t.h) * HD + col0);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
+        for (int q = 0; q < 4; ++q) {
           uint4 w;
-          w.x = pack_bf16(__uint_as_float(s[8 * q + 0]), __uint_as_float(s[8 * q + 1]));
-          w.y = pack_bf16(__uint_as_float(s[8 * q + 2]), __uint_as_float(s[8 * q + 3]));
-          w.z = pack_bf16(__uint_as_float(s[8 * q + 4]), __uint_as_float(s[8 * q + 5]));
-          w.w = pack_bf16(__uint_as_float(s[8 * q + 6]), __uint_as_float(s[8 * q + 7]));
+          w.x = pack_bf16(__uint_as_float(sv[8 * q + 0]), __uint_as_float(sv[8 * q + 1]));
+          w.y = pack_bf16(__uint_as_float(sv[8 * q + 2]), __uint_as_float(sv[8 * q + 3]));
+          w.z = pack_bf16(__uint_as_float(sv[8 * q + 4]), __uint_as_float(sv[8 * q + 5]));
+          w.w = pack_bf16(__uint_as_float(sv[8 * q + 6]), __uint_as_float(sv[8 * q + 7]));
           dst[q] = w;
         }
       }

@@ -136,7 +136,8 @@ static fc_status validate_config(const fc_config* c) {
 
 static void free_workspace(fc_handle* h) {
   fc::Workspace& w = h->ws;
-  void* ptrs[] = {w.q_buf, w.row_dst, w.imp_acc, w.items, w.sched, w.err, w.rope_cos, w.rope_sin};
+  void* ptrs[] = {w.q_buf, w.row_dst, w.imp_acc,  w.items,
+                  w.sched, w.err,     w.rope_cos, w.rope_sin};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   w = fc::Workspace{};

@@ -117,37 +117,47 @@ __global__ void __launch_bounds__(512) prep_kernel(StepShape s, const int32_t* _
       __syncthreads();
     }
   }
+  int* sseq = cnt + n2;   // [n2] sequence of each sorted slot
+  int* snq = sseq + n2;   // [n2] query tiles of each sorted slot
   for (int i = tid; i < n2; i += nt) {
-    int c = 0;
+    int c = 0, bq = 0, nqt = 0;
     if (i < s.B && (key[i] >> 63)) {
-      int bq = (int)(0xFFFFFFFFu - (unsigned)(key[i] & 0xFFFFFFFFull));
-      int n = cu_q[bq + 1] - cu_q[bq];
-      c = s.H * ((n + qtile - 1) / qtile);
+      bq = (int)(0xFFFFFFFFu - (unsigned)(key[i] & 0xFFFFFFFFull));
+      const int n = cu_q[bq + 1] - cu_q[bq];
+      nqt = (n + qtile - 1) / qtile;
+      c = s.H * nqt;
     }
     cnt[i] = c;
+    sseq[i] = bq;
+    snq[i] = nqt;
   }
   __syncthreads();
-  if (tid == 0) {  // serial exclusive scan; B <= 4096
-    int run = 0;
-    for (int i = 0; i < s.B; ++i) {
-      int c = cnt[i];
-      cnt[i] = run;
-      run += c;
+  if (tid < 32) {  // exclusive scan of cnt[0 .. B) by one warp
+    int carry = 0;
+    for (int base = 0; base < s.B; base += 32) {
+      const int i = base + tid;
+      const int v = i < s.B ? cnt[i] : 0;
+      int incl = v;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += u;
+      }
+      if (i < s.B) cnt[i] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    int total = min(run, max_items);
-    sched[0] = total;
-    sched[1] = 0;
+    if (tid == 0) {
+      sched[0] = min(carry, max_items);
+      sched[1] = 0;
+    }
   }
   __syncthreads();
   for (int i = 0; i < s.B; ++i) {
     if (!(key[i] >> 63)) break;
-    int bq = (int)(0xFFFFFFFFu - (unsigned)(key[i] & 0xFFFFFFFFull));
-    int n = cu_q[bq + 1] - cu_q[bq];
-    int nqt = (n + qtile - 1) / qtile;
-    int c = s.H * nqt;
-    int off = cnt[i];
+    const int bq = sseq[i], nqt = snq[i];
+    const int c = s.H * nqt;
+    const int off = cnt[i];
     for (int t = tid; t < c; t += nt) {
-      int hh = t / nqt, qt = t - hh * nqt;
+      const int hh = t / nqt, qt = t - hh * nqt;
       if (off + t < max_items) items[off + t] = WorkItem{bq, (qt << 8) | hh};
     }
   }
@@ -159,7 +169,7 @@ size_t prep_smem_bytes(int max_pos, int max_batch) {
   size_t bitmap = 2u * (size_t)((max_pos + 31) / 32) * sizeof(uint32_t);
   int n2 = 1;
   while (n2 < max_batch) n2 <<= 1;
-  size_t sortb = (size_t)n2 * (sizeof(unsigned long long) + sizeof(int));
+  size_t sortb = (size_t)n2 * (sizeof(unsigned long long) + 3 * sizeof(int));
   return bitmap > sortb ? bitmap : sortb;
 }
 
