@@ -13,20 +13,31 @@
 // summed, so the cache is scanned twice:
 //   pass 1: S = Q K^T per 128-key tile, row max m and sum l;
 //   pass 2: S = Q K^T again, P = 2^(S - m - log2 l) (final probabilities),
-//           O += P V and colsum(P) = ones * P, both on the tensor cores.
+//           O += P V on the tensor cores, column sums of P in registers.
 // Q arrives pre-scaled by log2(e)/sqrt(d) from the projection epilogue, so
 // scores are already in the exp2 domain.
+//
+// Operand placement: the tensor cores read their A operand from TMEM and only
+// K and V (the B operands) from shared memory.  Q is copied once per item from
+// shared memory into TMEM (tcgen05.cp); each tile's P is written (bf16) over the
+// S tile it came from (tcgen05.st), so P V of tile j and S of tile j+1 use
+// different buffers and the softmax never waits for the previous P V.
+//
+// TMEM columns: S/P buffer 0 [0,128), S/P buffer 1 [128,256), O [256,384),
+// Q [384,448).
 //
 // Roles (one CTA per SM, persistent over the work list):
 //   warp 0      TMA producer: Q tile, then K tiles (pass 1), then K and V
 //               tiles (pass 2) into a ring of four 32 KiB slots;
-//   warp 1      TMEM allocation and tcgen05.mma issue: S into two TMEM
-//               buffers, O and the column sums into their own TMEM columns;
+//   warp 1      TMEM allocation, Q copy and tcgen05.mma issue (S runs two
+//               tiles ahead of P V);
 //   warps 2-17  softmax: warp w owns TMEM lane quadrant w % 4 (32 query rows,
 //               one per thread) and a 32-column quarter (w - 2) / 4 of every
-//               128-column tile.  Four warps per scheduler keep the exp2
-//               pipe fed; the quarters' row statistics are merged once per
-//               item through shared memory.
+//               128-column tile.  The quarters' row statistics are merged once
+//               per item through shared memory; column sums are reduced across
+//               the warp with shuffles, across the four row quadrants in
+//               shared memory (2^-40 fixed point), and added to the global
+//               importance accumulator.
 #include <cuda_bf16.h>
 
 #include "fc_internal.h"
@@ -45,18 +56,16 @@ constexpr uint32_t HALF_BYTES = 128 * 128;       // 128 rows x 64 bf16
 constexpr uint32_t TILE_BYTES = 2 * HALF_BYTES;  // 128 rows x 128 bf16
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_SLOT = TILE_BYTES;
-constexpr uint32_t OFF_P = OFF_SLOT + SLOTS * TILE_BYTES;
-constexpr uint32_t OFF_ONES = OFF_P + TILE_BYTES;
-constexpr uint32_t ONES_BYTES = 2048;
-constexpr uint32_t OFF_STAT = OFF_ONES + ONES_BYTES;
+constexpr uint32_t OFF_CSACC = OFF_SLOT + SLOTS * TILE_BYTES;  // [2][128] int64 column sums
+constexpr uint32_t OFF_CSCNT = OFF_CSACC + 2 * 128 * 8;        // [2][PARTS] arrival counts
+constexpr uint32_t OFF_STAT = OFF_CSCNT + 64;
 constexpr uint32_t STAT_BYTES = 2 * PARTS * 2 * 128 * 4;  // [parity][part][m, l][row]
 constexpr uint32_t OFF_BARS = OFF_STAT + STAT_BYTES;
 // TMEM columns
-constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_CS = 384;
+constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_Q = 384;
 
-constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(128, 128, 0, 0);   // Q K^T, both K-major
+constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(128, 128, 0, 0);   // Q K^T, K K-major
 constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, 128, 0, 1);  // P V, V MN-major
-constexpr uint32_t IDESC_CS = ptx::idesc_bf16_f32(128, 128, 0, 1);  // ones P, P MN-major
 
 struct AttnParams {
   int H, max_T;
@@ -74,7 +83,7 @@ struct __align__(8) AttnBars {
   unsigned long long qfull, qfree;
   unsigned long long full[SLOTS], empty[SLOTS];
   unsigned long long sfull[2], sfree[2];
-  unsigned long long pready, pfree;
+  unsigned long long pready;
   unsigned long long ofull, ofree;
   unsigned long long statbar;
   unsigned long long drain;
@@ -121,26 +130,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7])
-      : "r"(taddr)
-      : "memory");
-}
-
 __global__ void __launch_bounds__(THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, AttnParams p) {
@@ -155,10 +144,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_items = p.sched[0];
 
-  // constant all-ones operand (8 rows x 128 columns, two 64-column atoms)
-  for (int i = tid; i < (int)(ONES_BYTES / 4); i += THREADS)
-    reinterpret_cast<uint32_t*>(smem + OFF_ONES)[i] = 0x3F803F80u;
-  fence_proxy_async_smem();
+  for (int i = tid; i < 2 * 128; i += THREADS)
+    reinterpret_cast<unsigned long long*>(smem + OFF_CSACC)[i] = 0ull;
+  if (tid < 2 * PARTS) reinterpret_cast<int*>(smem + OFF_CSCNT)[tid] = 0;
   if (tid == 0) {
     ptx::mbar_init(bar(bars->qfull), 1);
     ptx::mbar_init(bar(bars->qfree), 1);
@@ -171,7 +159,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       ptx::mbar_init(bar(bars->sfree[s]), SOFTMAX_WARPS);
     }
     ptx::mbar_init(bar(bars->pready), SOFTMAX_WARPS);
-    ptx::mbar_init(bar(bars->pfree), 1);
     ptx::mbar_init(bar(bars->ofull), 1);
     ptx::mbar_init(bar(bars->ofree), SOFTMAX_WARPS);
     ptx::mbar_init(bar(bars->statbar), SOFTMAX_WARPS);
@@ -251,13 +238,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t pcnt = 0;  // pready completions consumed
       uint32_t ic = 0;
       const uint32_t q_addr = base + OFF_Q;
-      const uint32_t p_addr = base + OFF_P;
-      const uint32_t ones_addr = base + OFF_ONES;
       auto slot_wait = [&](uint32_t idx) -> bool {
         return ptx::mbar_wait(bar(bars->full[idx % SLOTS]), (idx / SLOTS) & 1u, abort_flag);
       };
       auto slot_addr = [&](uint32_t idx) { return base + OFF_SLOT + (idx % SLOTS) * TILE_BYTES; };
-      // S[sb] = Q K^T for the K tile in production slot idx
+      // S[buffer] = Q K^T for the K tile in production slot idx (Q from TMEM)
       auto issue_s = [&](uint32_t idx) -> bool {
         const uint32_t sb = scnt & 1u;
         if (!ptx::mbar_wait(bar(bars->sfree[sb]), ((scnt >> 1) & 1u) ^ 1u, abort_flag)) return false;
@@ -267,7 +252,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * HALF_BYTES + (uint32_t)(k & 3) * 32;
-          ptx::mma_bf16_ss(tmem + TM_S0 + sb * 128, ptx::smem_desc(q_addr + off, 16, 1024),
+          ptx::mma_bf16_ts(tmem + TM_S0 + sb * 128, tmem + TM_Q + (uint32_t)(8 * k),
                            ptx::smem_desc(k_addr + off, 16, 1024), IDESC_S, k > 0 ? 1u : 0u);
         }
         ptx::mma_commit(bar(bars->sfull[sb]));
@@ -275,8 +260,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         ++scnt;
         return true;
       };
-      // O += P V and CS = ones P for the V tile in production slot idx
-      auto issue_pv = [&](uint32_t idx, bool first) -> bool {
+      // O += P V: P (bf16) sits in the first 64 columns of pass-2 tile j's S
+      // buffer, V in production slot idx
+      auto issue_pv = [&](uint32_t idx, uint32_t sb, bool first) -> bool {
         if (!ptx::mbar_wait(bar(bars->pready), pcnt & 1u, abort_flag)) return false;
         ++pcnt;
         if (!slot_wait(idx)) return false;
@@ -284,25 +270,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t v_addr = slot_addr(idx);
 #pragma unroll
         for (int k = 0; k < KT / 16; ++k) {
-          // A = P (K-major over keys); B = V (MN-major: d contiguous, keys are K)
-          const uint32_t poff = (uint32_t)(k >> 2) * HALF_BYTES + (uint32_t)(k & 3) * 32;
-          ptx::mma_bf16_ss(tmem + TM_O, ptx::smem_desc(p_addr + poff, 16, 1024),
+          // A = P from TMEM (keys are K); B = V (MN-major: d contiguous)
+          ptx::mma_bf16_ts(tmem + TM_O, tmem + TM_S0 + sb * 128 + (uint32_t)(8 * k),
                            ptx::smem_desc(v_addr + (uint32_t)k * 2048, HALF_BYTES, 1024), IDESC_PV,
                            (first && k == 0) ? 0u : 1u);
         }
-        if (p.want_imp) {
-#pragma unroll
-          for (int k = 0; k < QT / 16; ++k) {
-            // A = ones (rows alias one 8-row atom: SBO = 0); B = P^T (MN-major:
-            // keys contiguous, query rows are K)
-            const uint32_t aoff = (uint32_t)(k >> 2) * 1024 + (uint32_t)(k & 3) * 32;
-            ptx::mma_bf16_ss(tmem + TM_CS, ptx::smem_desc(ones_addr + aoff, 16, 0),
-                             ptx::smem_desc(p_addr + (uint32_t)k * 2048, HALF_BYTES, 1024),
-                             IDESC_CS, k > 0 ? 1u : 0u);
-          }
-        }
         ptx::mma_commit(bar(bars->empty[idx % SLOTS]));
-        ptx::mma_commit(bar(bars->pfree));
         return true;
       };
       for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
@@ -311,29 +284,41 @@ __global__ void __launch_bounds__(THREADS, 1)
           failed = true;
           break;
         }
+        ptx::tc_fence_after();
+        // Q: shared memory -> TMEM, one 16-column K slice per copy.  Copies and
+        // MMAs issued by this thread execute in order, so the copy cannot
+        // overtake the previous item's last S, and this item's S follows it.
+#pragma unroll
+        for (int k = 0; k < HD / 16; ++k) {
+          const uint32_t off = (uint32_t)(k >> 2) * HALF_BYTES + (uint32_t)(k & 3) * 32;
+          ptx::tmem_cp_128x256b(tmem + TM_Q + (uint32_t)(8 * k),
+                                ptx::smem_desc(q_addr + off, 16, 1024));
+        }
+        ptx::mma_commit(bar(bars->qfree));  // the shared-memory copy of Q is free again
         // pass 1: S tiles only
         for (int j = 0; j < t.ntiles && !failed; ++j)
           if (!issue_s(cons + (uint32_t)j)) failed = true;
         if (failed) break;
         const uint32_t base2 = cons + (uint32_t)t.ntiles;
+        const uint32_t sb0 = scnt & 1u;  // buffer of pass-2 tile 0
         // the previous item's O must have been read out before P V overwrites it
         if (!ptx::mbar_wait(bar(bars->ofree), (ic & 1u) ^ 1u, abort_flag)) {
           failed = true;
           break;
         }
+        // S runs two tiles ahead of P V; S[j+2] reuses tile j's buffer and is
+        // queued right after P V [j], which reads P[j] from that buffer
+        const int lead = t.ntiles < 2 ? t.ntiles : 2;
+        for (int j = 0; j < lead && !failed; ++j)
+          if (!issue_s(base2 + 2u * (uint32_t)j)) failed = true;
         for (int j = 0; j < t.ntiles && !failed; ++j) {
-          if (!issue_s(base2 + 2u * (uint32_t)j)) {
+          if (!issue_pv(base2 + 2u * (uint32_t)j + 1u, (sb0 + (uint32_t)j) & 1u, j == 0)) {
             failed = true;
             break;
           }
-          if (j == t.ntiles - 1) ptx::mma_commit(bar(bars->qfree));
-          if (j > 0 && !issue_pv(base2 + 2u * (uint32_t)(j - 1) + 1u, j == 1)) failed = true;
+          if (j + 2 < t.ntiles && !issue_s(base2 + 2u * (uint32_t)(j + 2))) failed = true;
         }
         if (failed) break;
-        if (!issue_pv(base2 + 2u * (uint32_t)(t.ntiles - 1) + 1u, t.ntiles == 1)) {
-          failed = true;
-          break;
-        }
         ptx::mma_commit(bar(bars->ofull));
         cons = base2 + 2u * (uint32_t)t.ntiles;
       }
@@ -353,30 +338,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int rl = quad * 32 + lane;  // query row inside the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const int col0 = CPW * part;      // first column of this warp in a tile
-    // this warp's 32 keys are 4 of the 8 16-byte chunks of one 64-key half of P
-    const uint32_t p_row = base + OFF_P + (uint32_t)(col0 >> 6) * HALF_BYTES + (uint32_t)rl * 128;
-    const uint32_t chunk0 = (uint32_t)((col0 & 63) >> 3);
     float* stat = reinterpret_cast<float*>(smem + OFF_STAT);  // [parity][part][m, l][row]
-    uint32_t scnt = 0, pfcnt = 0, ic = 0;
+    unsigned long long* cs_acc = reinterpret_cast<unsigned long long*>(smem + OFF_CSACC);
+    int* cs_cnt = reinterpret_cast<int*>(smem + OFF_CSCNT);
+    uint32_t scnt = 0, ic = 0;
 
-    // Column sums of the previous P tile (tile jt): every TMEM row of CS holds
-    // the same sums; warp (quad, part) takes columns col0 + 8*quad .. +7.
-    auto flush_colsum = [&](const Item& t, int jt) {
-      uint32_t r[8];
-      tmem_ld8(tmem + lane_off + TM_CS + (uint32_t)(col0 + 8 * quad), r);
-      ptx::tmem_wait_ld();
-      float v = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if (e == lane) v = __uint_as_float(r[e]);
-      const int key = jt * KT + col0 + 8 * quad + lane;
-      if (lane < 8 && key < t.L)
-        atomicAdd(&p.imp_acc[t.k0 + key], (unsigned long long)__double2ll_rn((double)v * kImpScale));
-    };
-    // This thread's 32 columns of the next S tile; the buffer is released at once.
-    auto load_s = [&](uint32_t (&sv)[32]) -> bool {
-      const uint32_t sb = scnt & 1u;
-      if (!ptx::mbar_wait(bar(bars->sfull[sb]), (scnt >> 1) & 1u, abort_flag)) return false;
+    // Load this thread's 32 columns of the next S tile and release the buffer;
+    // reports the buffer index and the parity of this use of it.
+    auto load_s = [&](uint32_t (&sv)[32], uint32_t& sb, uint32_t& par) -> bool {
+      sb = scnt & 1u;
+      par = (scnt >> 1) & 1u;
+      if (!ptx::mbar_wait(bar(bars->sfull[sb]), par, abort_flag)) return false;
       ptx::tc_fence_after();
       ptx::tmem_ld32(tmem + lane_off + TM_S0 + sb * 128 + (uint32_t)col0, sv);
       ptx::tmem_wait_ld();
@@ -386,14 +358,48 @@ __global__ void __launch_bounds__(THREADS, 1)
       ++scnt;
       return true;
     };
+    // Column sums of this warp's 32 rows x 32 columns (after the recursive
+    // halving lane l holds column l), then across the four row quadrants in
+    // shared memory; the last of the four warps adds them to the global
+    // accumulator.  Integer sums do not depend on arrival order.
+    auto add_colsums = [&](const Item& t, int jt, float (&v)[32]) {
+#pragma unroll
+      for (int st = 0; st < 5; ++st) {
+        const int o = 16 >> st;
+        const int hn = 16 >> st;
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < hn; ++i) {
+          const float send = upper ? v[i] : v[i + hn];
+          const float keep = upper ? v[i + hn] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      const int par = jt & 1;
+      unsigned long long* acc = cs_acc + par * 128 + col0;
+      atomicAdd(&acc[lane], (unsigned long long)__double2ll_rn((double)v[0] * kImpScale));
+      __threadfence_block();
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) last = atomicAdd(&cs_cnt[par * PARTS + part], 1) == 3;
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {
+        __threadfence_block();
+        const unsigned long long fx = atomicExch(&acc[lane], 0ull);
+        const int key = jt * KT + col0 + lane;
+        if (key < t.L && fx != 0ull) atomicAdd(&p.imp_acc[t.k0 + key], fx);
+        if (lane == 0) cs_cnt[par * PARTS + part] = 0;
+      }
+    };
 
     for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
       const Item t = load_item(p, it);
       uint32_t sv[32];
+      uint32_t sb, spar;
       // ---- pass 1: max and normaliser of this warp's 32-column quarter
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < t.ntiles; ++j) {
-        if (!load_s(sv)) {
+        if (!load_s(sv, sb, spar)) {
           failed = true;
           break;
         }
@@ -439,57 +445,38 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       // rows past the query tile's end get lse = +inf, i.e. P = 0
       const float lse = rl < t.nrows ? M + __log2f(Ls) : INFINITY;
-      // ---- pass 2: final probabilities -> P (smem); P V and colsum on the MMA
+      // ---- pass 2: final probabilities -> P (TMEM, over its S tile); column sums
       for (int j = 0; j < t.ntiles; ++j) {
-        if (!load_s(sv)) {
+        if (!load_s(sv, sb, spar)) {
           failed = true;
           break;
         }
         const int kmax = t.L - j * KT - col0;
-        uint32_t pk[16];
+        float pv[32];
         if (kmax >= 32) {
 #pragma unroll
-          for (int c = 0; c < 32; c += 2)
-            pk[c / 2] = pack_bf16(ex2(__uint_as_float(sv[c]) - lse),
-                                  ex2(__uint_as_float(sv[c + 1]) - lse));
+          for (int c = 0; c < 32; ++c) pv[c] = ex2(__uint_as_float(sv[c]) - lse);
         } else {
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float p0 = c < kmax ? ex2(__uint_as_float(sv[c]) - lse) : 0.f;
-            const float p1 = c + 1 < kmax ? ex2(__uint_as_float(sv[c + 1]) - lse) : 0.f;
-            pk[c / 2] = pack_bf16(p0, p1);
-          }
+          for (int c = 0; c < 32; ++c) pv[c] = c < kmax ? ex2(__uint_as_float(sv[c]) - lse) : 0.f;
         }
-        if (j > 0) {
-          // P buffer free (previous P V and colsum done): read that colsum
-          if (!ptx::mbar_wait(bar(bars->pfree), pfcnt & 1u, abort_flag)) {
-            failed = true;
-            break;
-          }
-          ++pfcnt;
-          ptx::tc_fence_after();
-          if (p.want_imp) flush_colsum(t, j - 1);
-        }
-        // 16-byte chunk index XOR (row & 7) is the 128-byte swizzle
+        uint32_t pk[16];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const uint32_t c16 = (chunk0 + (uint32_t)ch) ^ (uint32_t)(rl & 7);
-          st_shared_v4(p_row + (c16 << 4), pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2],
-                       pk[4 * ch + 3]);
+        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(pv[2 * c], pv[2 * c + 1]);
+        // every quarter of the tile must have been read before P overwrites it
+        if (!ptx::mbar_wait(bar(bars->sfree[sb]), spar, abort_flag)) {
+          failed = true;
+          break;
         }
-        fence_proxy_async_smem();
+        ptx::tc_fence_after();
+        ptx::tmem_st16(tmem + lane_off + TM_S0 + sb * 128 + (uint32_t)(col0 / 2), pk);
+        ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(bars->pready));
+        if (p.want_imp) add_colsums(t, j, pv);
       }
       if (failed) break;
-      if (!ptx::mbar_wait(bar(bars->pfree), pfcnt & 1u, abort_flag)) {
-        failed = true;
-        break;
-      }
-      ++pfcnt;
-      ptx::tc_fence_after();
-      if (p.want_imp) flush_colsum(t, t.ntiles - 1);
       // ---- O (already normalised) -> out
       if (!ptx::mbar_wait(bar(bars->ofull), ic & 1u, abort_flag)) {
         failed = true;
