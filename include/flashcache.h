@@ -175,6 +175,16 @@ FC_API fc_status fc_topk_tracked(fc_handle* h, void* stream, int batch, int tota
  */
 FC_API fc_status fc_get_error(fc_handle* h, int32_t* device_error_word);
 
+/*
+ * fc_selftest_wait_timeout — exercise the failure path of the bounded barrier
+ * waits.  Enqueues one CTA that waits on an mbarrier nothing arrives at, using
+ * the same bounded wait as the tensor-core kernels but a limit of `limit_us`
+ * microseconds (1 .. 2,000,000).  When the limit passes it sets
+ * FC_DEVERR_TIMEOUT in the handle's error word and returns; fc_get_error then
+ * reports FC_ERR_TIMEOUT and the CUDA context remains usable.
+ */
+FC_API fc_status fc_selftest_wait_timeout(fc_handle* h, void* stream, int limit_us);
+
 /* Number of kernels the last fc_step / fc_topk_tracked call enqueued (host). */
 FC_API int fc_last_launch_count(const fc_handle* h);
 

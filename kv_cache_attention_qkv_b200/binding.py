@@ -23,7 +23,8 @@ STATUS = {0: "FC_OK", -1: "FC_ERR_INVALID_ARG", -2: "FC_ERR_UNSUPPORTED", -3: "F
           -4: "FC_ERR_OOM", -5: "FC_ERR_DEVICE_CHECK", -6: "FC_ERR_TIMEOUT"}
 DEVERR = {0x01: "POS_RANGE", 0x02: "POS_DUP", 0x04: "SEQLENS", 0x08: "CAND", 0x10: "TIMEOUT"}
 EXPORTED = ("fc_create", "fc_step", "fc_topk_tracked", "fc_get_error", "fc_last_launch_count",
-            "fc_profile", "fc_profile_read", "fc_attention_noalloc", "fc_destroy", "fc_status_str")
+            "fc_profile", "fc_profile_read", "fc_attention_noalloc", "fc_selftest_wait_timeout",
+            "fc_destroy", "fc_status_str")
 PROFILE_SLOTS = ("prep", "qkv_rope_scatter", "attention", "importance_finalize", "topk")
 
 
@@ -68,6 +69,8 @@ def load_library(path: Optional[str] = None):
     lib.fc_profile.restype = c_int
     lib.fc_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(c_int)]
     lib.fc_profile_read.restype = c_int
+    lib.fc_selftest_wait_timeout.argtypes = [vp, vp, c_int]
+    lib.fc_selftest_wait_timeout.restype = c_int
     lib.fc_attention_noalloc.argtypes = [vp, c_int, c_int, c_int, c_int, vp, vp, vp, c_int, c_int,
                                          vp, vp, vp, vp]
     lib.fc_attention_noalloc.restype = c_int
@@ -193,6 +196,12 @@ class FlashCache:
         if st != 0:
             raise FlashCacheError(st, "fc_profile_read")
         return {name: (float(ms[i]), int(n[i])) for i, name in enumerate(PROFILE_SLOTS)}
+
+    def selftest_wait_timeout(self, limit_us: int, stream=None) -> None:
+        """Enqueue the bounded-wait self-test (see fc_selftest_wait_timeout)."""
+        st = self.lib.fc_selftest_wait_timeout(self._h, _stream_handle(stream), int(limit_us))
+        if st != 0:
+            raise FlashCacheError(st, "fc_selftest_wait_timeout")
 
     @property
     def last_launch_count(self) -> int:

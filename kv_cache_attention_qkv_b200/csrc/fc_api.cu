@@ -344,6 +344,17 @@ fc_status fc_get_error(fc_handle* h, int32_t* device_error_word) {
 
 int fc_last_launch_count(const fc_handle* h) { return h ? h->last_launches : 0; }
 
+fc_status fc_selftest_wait_timeout(fc_handle* h, void* stream, int limit_us) {
+  if (!h || limit_us < 1 || limit_us > 2000000) return FC_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return FC_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  h->last_stream = st;
+  h->last_launches = 0;
+  if (fc::launch_selftest_wait_timeout(h, st, limit_us) != cudaSuccess) return FC_ERR_CUDA;
+  h->last_launches = 1;
+  return FC_OK;
+}
+
 fc_status fc_profile(fc_handle* h, int enable) {
   if (!h || (enable != 0 && enable != 1)) return FC_ERR_INVALID_ARG;
   if (cudaSetDevice(h->device) != cudaSuccess) return FC_ERR_CUDA;

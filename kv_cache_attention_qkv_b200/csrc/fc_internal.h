@@ -92,6 +92,7 @@ cudaError_t launch_topk(const fc_handle* h, cudaStream_t st, int B, int S, const
                         const int32_t* cu_k, const int32_t* cand_lo, const int32_t* cand_hi,
                         const int32_t* k_per_seq, int k, int32_t* tracked);
 
+cudaError_t launch_selftest_wait_timeout(const fc_handle* h, cudaStream_t st, int limit_us);
 size_t qkv_tc_smem_bytes();
 size_t attn_tc_smem_bytes();
 bool encode_kv_3d(CUtensorMap* tm, const void* cache, int S, int H);

@@ -193,3 +193,19 @@ def test_device_checks_set_error_word(bad):
             row = inp.seq_slice_k(0).start + inp.q_pos[4]
             np.testing.assert_array_equal(k_now[row], prior_k[row])
     assert tl.run_gpu(workloads.generate("small_varlen"), layer=gpu["layer"])["err"] == 0
+
+
+def test_bounded_wait_times_out_and_context_stays_usable():
+    """A barrier that never completes turns into FC_ERR_TIMEOUT, not a hang;
+    the next step on the same handle is correct."""
+    from kv_cache_attention_qkv_b200.binding import describe_error_word
+
+    inp = workloads.generate("small_varlen")
+    dev = tl.upload(inp)
+    layer = tl.make_layer(inp, dev["w"])
+    layer.selftest_wait_timeout(50_000)  # 50 ms
+    word = layer.get_error()
+    assert "TIMEOUT" in describe_error_word(word)
+    gpu = tl.run_gpu(inp, layer=layer, dev=dev)
+    assert gpu["err"] == 0
+    tl.compare_step(inp, gpu, tl.run_oracle(inp), range(inp.batch))
