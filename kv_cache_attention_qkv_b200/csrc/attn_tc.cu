@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   auto bar = [](unsigned long long& b) { return ptx::smem_u32(&b); };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_items = p.sched[0];
+  ptx::griddep_launch_dependents();
 
   for (int i = tid; i < 2 * 128; i += THREADS)
     reinterpret_cast<unsigned long long*>(smem + OFF_CSACC)[i] = 0ull;
@@ -178,6 +178,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   bool failed = false;
+  // the work list, Q and the refreshed cache come from the preceding kernels
+  ptx::griddep_wait();
+  const int n_items = p.sched[0];
 
   if (warp == 0) {
     if (lane == 0) {
@@ -536,7 +539,8 @@ cudaError_t launch_attn_tc(const fc_handle* h, cudaStream_t st, const StepShape&
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<<<h->num_sms, THREADS, smem, st>>>(h->tm_q, tm_k, tm_v, p);
+  e = launch_pdl(attn_tc_kernel, dim3(h->num_sms), dim3(THREADS), smem, st, h->tm_q, tm_k, tm_v, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

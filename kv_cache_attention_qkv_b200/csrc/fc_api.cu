@@ -213,7 +213,7 @@ fc_status fc_create(const fc_config* cfg, const void* w_qkv, fc_handle** out) {
        cudaMemset(w.row_dst, 0xFF, (size_t)cfg->max_total_q * sizeof(int32_t)) == cudaSuccess;
   if (ok && h->tc_gemm)
     ok = fc::encode_bf16_2d(&h->tm_w, w_qkv, (uint64_t)3 * H * d, (uint64_t)cfg->hidden,
-                            (uint64_t)cfg->hidden * 2, 256, 64);
+                            (uint64_t)cfg->hidden * 2, fc::kQkvWBoxRows, 64);
   if (ok && h->tc_attn)
     ok = fc::encode_bf16_2d(&h->tm_q, w.q_buf, (uint64_t)cfg->max_total_q * H, (uint64_t)d,
                             (uint64_t)d * 2, 128, 64) &&
@@ -268,7 +268,7 @@ fc_status fc_step(fc_handle* h, void* stream, int batch, const void* x, const in
   if (h->tc_gemm) {
     CUtensorMap tm_x;
     if (!fc::encode_bf16_2d(&tm_x, x, (uint64_t)total_q, (uint64_t)c.hidden,
-                            (uint64_t)c.hidden * 2, 128, 64))
+                            (uint64_t)c.hidden * 2, fc::kQkvXBoxRows, 64))
       return FC_ERR_CUDA;
     ProfScope ps(h, st, 1);
     e = fc::launch_qkv_tc(h, st, s, tm_x, q_pos, k_cache, v_cache);

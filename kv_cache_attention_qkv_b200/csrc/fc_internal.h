@@ -15,6 +15,11 @@ namespace fc {
 constexpr int kTcQTile = 128;
 constexpr int kSimtQTile = 16;
 
+// TMA boxes of the tensor-core projection (rows x 64 bf16 columns): each CTA
+// of a pair loads 128 rows of X and 128 rows (half the 256-row tile) of W.
+constexpr int kQkvXBoxRows = 128;
+constexpr int kQkvWBoxRows = 128;
+
 // Importance is accumulated in fixed point (int64, 2^-40 units) so that the
 // sum over heads and query tiles is exact and independent of the order in
 // which work items finish.  One column sum is at most kSimtQTile..128 and a
@@ -69,6 +74,25 @@ struct fc_handle {
 };
 
 namespace fc {
+
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while the previous kernel of the stream is still running; it must call
+// griddepcontrol.wait before touching that kernel's outputs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 // ---- launchers (each returns the CUDA error of its launch) -----------------
 cudaError_t launch_prep(const fc_handle* h, cudaStream_t st, const StepShape& s,

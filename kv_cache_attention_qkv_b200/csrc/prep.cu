@@ -7,6 +7,7 @@
 // Flash-Cache paragraph).  Rows whose position is outside the sequence, or
 // shared with another row of the same sequence, get -1 and are never written.
 #include "fc_internal.h"
+#include "ptx.cuh"
 
 namespace fc {
 namespace {
@@ -36,6 +37,9 @@ __global__ void __launch_bounds__(512) prep_kernel(StepShape s, const int32_t* _
   extern __shared__ uint32_t smem[];
   const int b = blockIdx.x;
   const int tid = threadIdx.x, nt = blockDim.x;
+  // the projection may start its main loop now; it waits for this grid before
+  // its epilogue reads the row map
+  ptx::griddep_launch_dependents();
 
   if (b < s.B) {
     const bool ok = seq_ok(cu_q, cu_k, b, s.B, s.T, s.S, s.max_pos, s.max_seqlen_q);

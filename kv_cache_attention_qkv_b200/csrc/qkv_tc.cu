@@ -10,13 +10,18 @@
 //     attention reads it, else [T, H, d]),
 //   k, v (bf16, round to nearest even) -> cache row cu_seqlens_k[b] + q_pos[r].
 //
-// Structure (one CTA per SM, persistent over output tiles):
-//   warp 0     TMA producer: X and W tiles (64-wide K slices, 128-byte swizzle)
-//              into a 4-stage shared-memory ring;
-//   warp 1     allocates 512 TMEM columns and issues tcgen05.mma (M=128,
-//              N=256, K=16) into one of two TMEM accumulators;
-//   warps 2-5  epilogue: tcgen05.ld of its 32-row quadrant, RoPE, stores,
-//              while the MMA warp already fills the other accumulator.
+// Structure: CTA pairs (clusters of two), each pair persistent over 256 x 256
+// output tiles; one tcgen05.mma.cta_group::2 (M=256, N=256, K=16) covers the
+// pair, each CTA holding 128 rows of X and 128 rows of W per stage, so each SM
+// streams half of the W tile through its shared memory.
+//   warp 0     TMA producer (both CTAs): X and W slices (64 wide, 128-byte
+//              swizzle) into a 6-stage ring; completion is counted on the
+//              leader CTA's barrier;
+//   warp 1     allocates 512 TMEM columns (pair allocation); in the leader CTA
+//              it issues the MMAs into one of two TMEM accumulators and
+//              releases stages and accumulators to both CTAs (multicast commit);
+//   warps 2-5  epilogue (both CTAs): tcgen05.ld of its 32-row quadrant, RoPE,
+//              stores, while the MMA warp already fills the other accumulator.
 #include <cuda_bf16.h>
 
 #include "fc_internal.h"
@@ -25,13 +30,17 @@
 namespace fc {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128;                         // rows of X per CTA
+constexpr int PM = 256;                         // rows per pair tile
+constexpr int BN = 256, BK = 64, STAGES = 6;
 constexpr int HD = 128;                         // head_dim of this path
 constexpr uint32_t A_BYTES = BM * BK * 2;       // 16 KiB
-constexpr uint32_t B_BYTES = BN * BK * 2;       // 32 KiB
+constexpr uint32_t B_BYTES = (BN / 2) * BK * 2; // 16 KiB: this CTA's half of the W tile
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int GROUP_M = 8;                      // tile raster: groups of 8 row blocks
-constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, BN, 0, 0);
+static_assert(kQkvXBoxRows == BM && kQkvWBoxRows == BN / 2,
+              "the host's TMA boxes must match the per-CTA tiles");
+constexpr int GROUP_M = 8;                      // tile raster: groups of 8 pair row blocks
+constexpr uint32_t IDESC = ptx::idesc_bf16_f32(PM, BN, 0, 0);
 constexpr int THREADS = 192;
 
 struct QkvParams {
@@ -100,6 +109,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   auto sB = [&](int s) { return base + s * STAGE_BYTES + A_BYTES; };
   auto bar = [](unsigned long long& b) { return ptx::smem_u32(&b); };
 
+  ptx::griddep_launch_dependents();
+  const uint32_t rank = ptx::cluster_ctarank();  // 0 = leader of the pair
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(bar(bars->full[s]), 1);
@@ -107,7 +120,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(bar(bars->tfull[a]), 1);
-      ptx::mbar_init(bar(bars->tempty[a]), 4);
+      ptx::mbar_init(bar(bars->tempty[a]), 8);  // 4 epilogue warps in each CTA
     }
     ptx::mbar_init(bar(bars->drain), 1);
     bars->abort_flag = 0;
@@ -116,11 +129,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     ptx::prefetch_tmap(&tm_w);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(ptx::smem_u32(&bars->tmem_base), 512);
-    ptx::tmem_relinquish();
+    ptx::tmem_alloc_pair(ptx::smem_u32(&bars->tmem_base), 512);
+    ptx::tmem_relinquish_pair();
   }
   ptx::tc_fence_before();
   __syncthreads();
+  ptx::cluster_sync();  // both CTAs' barriers exist before any cross-CTA traffic
   ptx::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   bool failed = false;
@@ -132,7 +146,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t phase = 0;
       int issued_phase[STAGES];
       for (int s = 0; s < STAGES; ++s) issued_phase[s] = -1;
-      for (int t = blockIdx.x; t < p.num_tiles && !failed; t += gridDim.x) {
+      for (int t = pair; t < p.num_tiles && !failed; t += npairs) {
         int m, n;
         tile_coords(t, p.num_m, p.num_n, m, n);
         for (int kb = 0; kb < p.num_k; ++kb) {
@@ -140,9 +154,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             failed = true;
             break;
           }
-          ptx::mbar_arrive_expect_tx(bar(bars->full[stage]), STAGE_BYTES);
-          ptx::tma_load_2d(sA(stage), &tm_x, kb * BK, m * BM, bar(bars->full[stage]));
-          ptx::tma_load_2d(sB(stage), &tm_w, kb * BK, n * BN, bar(bars->full[stage]));
+          // the leader's barrier counts both CTAs' bytes
+          if (leader) ptx::mbar_arrive_expect_tx(bar(bars->full[stage]), 2 * STAGE_BYTES);
+          const uint32_t lbar = ptx::mapa_shared(bar(bars->full[stage]), 0);
+          ptx::tma_load_2d_pair(sA(stage), &tm_x, kb * BK, m * PM + (int)rank * BM, lbar);
+          ptx::tma_load_2d_pair(sB(stage), &tm_w, kb * BK, n * BN + (int)rank * (BN / 2), lbar);
           issued_phase[stage] = (int)phase;
           if (++stage == STAGES) {
             stage = 0;
@@ -150,8 +166,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      if (failed) {
-        // let the copies already in flight land before the CTA exits
+      if (failed && leader) {
+        // let the copies already in flight land before the CTA exits (the
+        // leader's barriers also count the other CTA's copies)
         *abort_flag = 1;
         for (int s = 0; s < STAGES; ++s)
           if (issued_phase[s] >= 0) {
@@ -163,12 +180,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (leader CTA only)
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
-      for (int t = blockIdx.x; t < p.num_tiles && !failed; t += gridDim.x, ++it) {
+      for (int t = pair; t < p.num_tiles && !failed; t += npairs, ++it) {
         const int a = it & 1;
         const uint32_t u = (uint32_t)(it >> 1);
         if (!ptx::mbar_wait(bar(bars->tempty[a]), (u & 1u) ^ 1u, abort_flag)) {
@@ -187,20 +204,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t ad = ptx::smem_desc(sA(stage) + k * 32, 16, 1024);
             const uint64_t bd = ptx::smem_desc(sB(stage) + k * 32, 16, 1024);
-            ptx::mma_bf16_ss(d, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
+            ptx::mma_bf16_ss_pair(d, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
           }
-          ptx::mma_commit(bar(bars->empty[stage]));
+          ptx::mma_commit_pair_mc(bar(bars->empty[stage]), 0x3);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (failed) break;
-        ptx::mma_commit(bar(bars->tfull[a]));
+        ptx::mma_commit_pair_mc(bar(bars->tfull[a]), 0x3);
       }
       if (failed) {
         *abort_flag = 1;
-        ptx::mma_commit(bar(bars->drain));
+        ptx::mma_commit_pair_mc(bar(bars->drain), 0x1);
         const unsigned long long t0 = ptx::globaltimer();
         while (!ptx::mbar_try_wait(bar(bars->drain), 0u) &&
                ptx::globaltimer() - t0 < ptx::kWaitLimitNs) {
@@ -212,7 +229,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int quad = warp & 3;
     const int half = HD / 2;
     int it = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++it) {
+    ptx::griddep_wait();  // the row map comes from the preparation kernel
+    const uint32_t tempty_leader0 = ptx::mapa_shared(bar(bars->tempty[0]), 0);
+    const uint32_t tempty_leader1 = ptx::mapa_shared(bar(bars->tempty[1]), 0);
+    for (int t = pair; t < p.num_tiles; t += npairs, ++it) {
       int m, n;
       tile_coords(t, p.num_m, p.num_n, m, n);
       const int a = it & 1;
@@ -223,7 +243,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       }
       ptx::tc_fence_after();
-      const int row = m * BM + quad * 32 + lane;
+      const int row = m * PM + (int)rank * BM + quad * 32 + lane;
       const bool in = row < p.T;
       const int dst = in ? p.row_dst[row] : -1;
       const bool valid = dst >= 0 && dst < p.S;
@@ -282,16 +302,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(bars->tempty[a]));
+      if (lane == 0) ptx::mbar_arrive_cluster(a ? tempty_leader1 : tempty_leader0);
     }
   }
 
   __syncwarp();
   ptx::tc_fence_before();
   __syncthreads();
+  ptx::cluster_sync();  // the pair's MMAs and cross-CTA arrivals are all done
   ptx::tc_fence_after();
   if (tid == 0 && bars->abort_flag) atomicOr(p.err, FC_DEVERR_TIMEOUT);
-  if (warp == 1) ptx::tmem_dealloc(tmem, 512);
+  if (warp == 1) ptx::tmem_dealloc_pair(tmem, 512);
 }
 
 }  // namespace
@@ -306,7 +327,7 @@ cudaError_t launch_qkv_tc(const fc_handle* h, cudaStream_t st, const StepShape& 
   p.S = s.S;
   p.D = s.D;
   p.H = s.H;
-  p.num_m = (s.T + BM - 1) / BM;
+  p.num_m = (s.T + PM - 1) / PM;
   p.num_n = 3 * s.H * HD / BN;
   p.num_tiles = p.num_m * p.num_n;
   p.num_k = s.D / BK;
@@ -330,8 +351,34 @@ cudaError_t launch_qkv_tc(const fc_handle* h, cudaStream_t st, const StepShape& 
   cudaError_t e = cudaFuncSetAttribute(qkv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  const int grid = p.num_tiles < h->num_sms ? p.num_tiles : h->num_sms;
-  qkv_tc_kernel<<<grid, THREADS, smem, st>>>(tm_x, h->tm_w, p);
+  int pairs = h->num_sms / 2;
+  if (p.num_tiles < pairs) pairs = p.num_tiles;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int max_clusters = 0;
+  cfg.numAttrs = 1;  // occupancy query with the cluster shape only
+  const bool occ_ok = cudaOccupancyMaxActiveClusters(&max_clusters, qkv_tc_kernel, &cfg) == cudaSuccess;
+  cfg.numAttrs = 2;
+  if (occ_ok &&
+      max_clusters > 0 && max_clusters < pairs) {
+    pairs = max_clusters;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+  }
+  cudaGetLastError();
+  e = cudaLaunchKernelEx(&cfg, qkv_tc_kernel, tm_x, h->tm_w, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -12,12 +12,15 @@
 // the kept set is sorted by (score desc, position asc).  The result does not
 // depend on thread timing.
 #include "fc_internal.h"
+#include "ptx.cuh"
 
 namespace fc {
 namespace {
 
 __global__ void importance_finalize(int S, unsigned long long* __restrict__ acc,
                                     float* __restrict__ imp, int accumulate) {
+  ptx::griddep_launch_dependents();
+  ptx::griddep_wait();
   for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < S; j += gridDim.x * blockDim.x) {
     const double v = (double)(long long)acc[j] * kImpInvScale;
     const float f = (float)v;
@@ -47,6 +50,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(
 
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t* row = tracked + (size_t)b * k;
+  ptx::griddep_wait();  // importance comes from the preceding step
 
   const int k0 = cu_k[b], k1 = cu_k[b + 1];
   const int lo = cand_lo[b], hi = cand_hi[b];
@@ -179,15 +183,18 @@ cudaError_t launch_importance_finalize(const fc_handle* h, cudaStream_t st, int 
   if (S <= 0) return cudaSuccess;
   int blocks = (S + 255) / 256;
   if (blocks > h->num_sms * 8) blocks = h->num_sms * 8;
-  importance_finalize<<<blocks, 256, 0, st>>>(S, h->ws.imp_acc, importance, accumulate);
+  cudaError_t e = launch_pdl(importance_finalize, dim3(blocks), dim3(256), 0, st, S, h->ws.imp_acc,
+                             importance, accumulate);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_topk(const fc_handle* h, cudaStream_t st, int B, int S, const float* importance,
                         const int32_t* cu_k, const int32_t* cand_lo, const int32_t* cand_hi,
                         const int32_t* k_per_seq, int k, int32_t* tracked) {
-  topk_kernel<<<B, TK_THREADS, 0, st>>>(B, importance, cu_k, cand_lo, cand_hi, k_per_seq, k,
-                                        tracked, h->ws.err, S, h->cfg.max_pos);
+  cudaError_t e = launch_pdl(topk_kernel, dim3(B), dim3(TK_THREADS), 0, st, B, importance, cu_k,
+                             cand_lo, cand_hi, k_per_seq, k, tracked, h->ws.err, S, h->cfg.max_pos);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
