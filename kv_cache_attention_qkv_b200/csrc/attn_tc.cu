@@ -21,7 +21,9 @@
 // K and V (the B operands) from shared memory.  Q is copied once per item from
 // shared memory into TMEM (tcgen05.cp); each tile's P is written (bf16) over the
 // S tile it came from (tcgen05.st), so P V of tile j and S of tile j+1 use
-// different buffers and the softmax never waits for the previous P V.
+// different buffers and the softmax never waits for the previous P V.  Keys
+// 64h..64h+63 of a tile go, packed, to columns 64h..64h+31 of its buffer: every
+// softmax warp overwrites only columns it has already read itself.
 //
 // TMEM columns: S/P buffer 0 [0,128), S/P buffer 1 [128,256), O [256,384),
 // Q [384,448).
@@ -31,9 +33,12 @@
 //               tiles (pass 2) into a ring of four 32 KiB slots;
 //   warp 1      TMEM allocation, Q copy and tcgen05.mma issue (S runs two
 //               tiles ahead of P V);
-//   warps 2-17  softmax: warp w owns TMEM lane quadrant w % 4 (32 query rows,
-//               one per thread) and a 32-column quarter (w - 2) / 4 of every
-//               128-column tile.  The quarters' row statistics are merged once
+//   warps 2-17  softmax, two groups of eight that take S tiles alternately
+//               (group g owns the tiles in TMEM buffer g), so one group's
+//               exp2 work overlaps the other's hand-off to the tensor cores.
+//               In a group, warp w owns TMEM lane quadrant w % 4 (32 query
+//               rows, one per thread) and one 64-column half of the tile.
+//               Row statistics of the four (group, half) parts are merged once
 //               per item through shared memory; column sums are reduced across
 //               the warp with shuffles, across the four row quadrants in
 //               shared memory (2^-40 fixed point), and added to the global
@@ -48,16 +53,19 @@ namespace {
 
 constexpr int QT = 128, KT = 128, HD = 128;
 constexpr int SLOTS = 4;
-constexpr int SOFTMAX_WARPS = 16;
-constexpr int PARTS = 4;         // column quarters per row quadrant
-constexpr int CPW = KT / PARTS;  // columns per softmax warp
+constexpr int SOFTMAX_WARPS = 16;  // two groups of 8
+constexpr int PARTS = 4;           // (group, column half) partial row statistics
+constexpr int CPW = KT / 2;        // columns per softmax warp and tile
 constexpr int THREADS = 64 + 32 * SOFTMAX_WARPS;
 constexpr uint32_t HALF_BYTES = 128 * 128;       // 128 rows x 64 bf16
 constexpr uint32_t TILE_BYTES = 2 * HALF_BYTES;  // 128 rows x 128 bf16
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_SLOT = TILE_BYTES;
-constexpr uint32_t OFF_CSACC = OFF_SLOT + SLOTS * TILE_BYTES;  // [2][128] int64 column sums
-constexpr uint32_t OFF_CSCNT = OFF_CSACC + 2 * 128 * 8;        // [2][PARTS] arrival counts
+// column sums, int64 [group][tile parity within the group][128]: a warp can
+// reach its group's next tile before the quadrant that flushes this one has
+// finished, but not the tile after (that S waits for this warp's own P).
+constexpr uint32_t OFF_CSACC = OFF_SLOT + SLOTS * TILE_BYTES;
+constexpr uint32_t OFF_CSCNT = OFF_CSACC + 4 * 128 * 8;  // [group][parity][half] arrival counts
 constexpr uint32_t OFF_STAT = OFF_CSCNT + 64;
 constexpr uint32_t STAT_BYTES = 2 * PARTS * 2 * 128 * 4;  // [parity][part][m, l][row]
 constexpr uint32_t OFF_BARS = OFF_STAT + STAT_BYTES;
@@ -83,7 +91,7 @@ struct __align__(8) AttnBars {
   unsigned long long qfull, qfree;
   unsigned long long full[SLOTS], empty[SLOTS];
   unsigned long long sfull[2], sfree[2];
-  unsigned long long pready;
+  unsigned long long pready[2];
   unsigned long long ofull, ofree;
   unsigned long long statbar;
   unsigned long long drain;
@@ -110,13 +118,25 @@ __device__ __forceinline__ Item load_item(const AttnParams& p, int it) {
   return r;
 }
 
+// Tiled 3-D TMA load with an L2 eviction-priority policy (createpolicy).
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, int x, int y,
-                                            int z, uint32_t bar) {
+                                            int z, uint32_t bar, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(policy)
       : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -144,9 +164,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   ptx::griddep_launch_dependents();
 
-  for (int i = tid; i < 2 * 128; i += THREADS)
+  for (int i = tid; i < 4 * 128; i += THREADS)
     reinterpret_cast<unsigned long long*>(smem + OFF_CSACC)[i] = 0ull;
-  if (tid < 2 * PARTS) reinterpret_cast<int*>(smem + OFF_CSCNT)[tid] = 0;
+  if (tid < 8) reinterpret_cast<int*>(smem + OFF_CSCNT)[tid] = 0;
   if (tid == 0) {
     ptx::mbar_init(bar(bars->qfull), 1);
     ptx::mbar_init(bar(bars->qfree), 1);
@@ -156,9 +176,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(bar(bars->sfull[s]), 1);
-      ptx::mbar_init(bar(bars->sfree[s]), SOFTMAX_WARPS);
+      ptx::mbar_init(bar(bars->sfree[s]), SOFTMAX_WARPS / 2);  // the owning group
+      ptx::mbar_init(bar(bars->pready[s]), SOFTMAX_WARPS / 2);
     }
-    ptx::mbar_init(bar(bars->pready), SOFTMAX_WARPS);
     ptx::mbar_init(bar(bars->ofull), 1);
     ptx::mbar_init(bar(bars->ofree), SOFTMAX_WARPS);
     ptx::mbar_init(bar(bars->statbar), SOFTMAX_WARPS);
@@ -190,13 +210,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int s = 0; s < SLOTS; ++s) issued_phase[s] = -1;
       int q_issued_phase = -1;
       uint32_t ic = 0;
-      auto load_tile = [&](const CUtensorMap* tm, int h, int row) -> bool {
+      // K is read again by pass 2 of the same item: keep it in L2 over V,
+      // which (like the second read of K) is read once and streams through.
+      const uint64_t pol_keep = policy_evict_last(), pol_stream = policy_evict_first();
+      auto load_tile = [&](const CUtensorMap* tm, int h, int row, uint64_t pol) -> bool {
         const uint32_t s = prod % SLOTS, ph = (prod / SLOTS) & 1u;
         if (!ptx::mbar_wait(bar(bars->empty[s]), ph ^ 1u, abort_flag)) return false;
         const uint32_t dst = base + OFF_SLOT + s * TILE_BYTES;
         ptx::mbar_arrive_expect_tx(bar(bars->full[s]), TILE_BYTES);
-        tma_load_3d(dst, tm, 0, h, row, bar(bars->full[s]));
-        tma_load_3d(dst + HALF_BYTES, tm, 64, h, row, bar(bars->full[s]));
+        tma_load_3d(dst, tm, 0, h, row, bar(bars->full[s]), pol);
+        tma_load_3d(dst + HALF_BYTES, tm, 64, h, row, bar(bars->full[s]), pol);
         issued_phase[s] = (int)ph;
         ++prod;
         return true;
@@ -212,10 +235,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         ptx::tma_load_2d(base + OFF_Q, &tm_q, 0, qrow, bar(bars->qfull));
         ptx::tma_load_2d(base + OFF_Q + HALF_BYTES, &tm_q, 64, qrow, bar(bars->qfull));
         q_issued_phase = (int)(ic & 1u);
-        for (int j = 0; j < t.ntiles && !failed; ++j)
-          if (!load_tile(&tm_k, t.h, t.k0 + j * KT)) failed = true;
         for (int j = 0; j < t.ntiles && !failed; ++j) {
-          if (!load_tile(&tm_k, t.h, t.k0 + j * KT) || !load_tile(&tm_v, t.h, t.k0 + j * KT))
+          if (!load_tile(&tm_k, t.h, t.k0 + j * KT, pol_keep)) failed = true;
+        }
+        for (int j = 0; j < t.ntiles && !failed; ++j) {
+          if (!load_tile(&tm_k, t.h, t.k0 + j * KT, pol_stream) ||
+              !load_tile(&tm_v, t.h, t.k0 + j * KT, pol_stream))
             failed = true;
         }
       }
@@ -238,7 +263,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ---------------------------------------------------------- MMA issuer
       uint32_t cons = 0;  // slot consumption index base (production order)
       uint32_t scnt = 0;  // S tiles issued
-      uint32_t pcnt = 0;  // pready completions consumed
+      uint32_t pcnt[2] = {0u, 0u};  // pready completions consumed, per buffer
       uint32_t ic = 0;
       const uint32_t q_addr = base + OFF_Q;
       auto slot_wait = [&](uint32_t idx) -> bool {
@@ -263,18 +288,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         ++scnt;
         return true;
       };
-      // O += P V: P (bf16) sits in the first 64 columns of pass-2 tile j's S
-      // buffer, V in production slot idx
+      // O += P V: P (bf16) of pass-2 tile j sits in columns 0-31 (keys 0-63)
+      // and 64-95 (keys 64-127) of its S buffer, V in production slot idx
       auto issue_pv = [&](uint32_t idx, uint32_t sb, bool first) -> bool {
-        if (!ptx::mbar_wait(bar(bars->pready), pcnt & 1u, abort_flag)) return false;
-        ++pcnt;
+        if (!ptx::mbar_wait(bar(bars->pready[sb]), pcnt[sb] & 1u, abort_flag)) return false;
+        ++pcnt[sb];
         if (!slot_wait(idx)) return false;
         ptx::tc_fence_after();
         const uint32_t v_addr = slot_addr(idx);
 #pragma unroll
         for (int k = 0; k < KT / 16; ++k) {
           // A = P from TMEM (keys are K); B = V (MN-major: d contiguous)
-          ptx::mma_bf16_ts(tmem + TM_O, tmem + TM_S0 + sb * 128 + (uint32_t)(8 * k),
+          ptx::mma_bf16_ts(tmem + TM_O, tmem + TM_S0 + sb * 128 + (uint32_t)(64 * (k >> 2) + 8 * (k & 3)),
                            ptx::smem_desc(v_addr + (uint32_t)k * 2048, HALF_BYTES, 1024), IDESC_PV,
                            (first && k == 0) ? 0u : 1u);
         }
@@ -336,38 +361,40 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ---------------------------------------------------------- softmax warps
+    const int sw = warp - 2;
+    const int grp = sw >> 3;            // owns the S tiles in TMEM buffer grp
+    const int hf = (sw >> 2) & 1;       // 64-column half of every tile
     const int quad = warp & 3;
-    const int part = (warp - 2) >> 2;
-    const int rl = quad * 32 + lane;  // query row inside the tile = TMEM lane
+    const int part = grp * 2 + hf;      // index of this warp's partial statistics
+    const int rl = quad * 32 + lane;    // query row inside the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const int col0 = CPW * part;      // first column of this warp in a tile
+    const int col0 = CPW * hf;
+    const uint32_t sbuf = tmem + TM_S0 + (uint32_t)grp * 128;
     float* stat = reinterpret_cast<float*>(smem + OFF_STAT);  // [parity][part][m, l][row]
-    unsigned long long* cs_acc = reinterpret_cast<unsigned long long*>(smem + OFF_CSACC);
-    int* cs_cnt = reinterpret_cast<int*>(smem + OFF_CSCNT);
-    uint32_t scnt = 0, ic = 0;
+    unsigned long long* cs_base =
+        reinterpret_cast<unsigned long long*>(smem + OFF_CSACC) + grp * 256 + col0;
+    int* cnt_base = reinterpret_cast<int*>(smem + OFF_CSCNT) + grp * 4 + hf;
+    uint32_t gs = 0, ic = 0;  // global S tile index (same sequence as the MMA warp)
 
-    // Load this thread's 32 columns of the next S tile and release the buffer;
-    // reports the buffer index and the parity of this use of it.
-    auto load_s = [&](uint32_t (&sv)[32], uint32_t& sb, uint32_t& par) -> bool {
-      sb = scnt & 1u;
-      par = (scnt >> 1) & 1u;
-      if (!ptx::mbar_wait(bar(bars->sfull[sb]), par, abort_flag)) return false;
+    // This thread's 64 columns of S tile `s` (buffer grp); the buffer is
+    // released to the MMA warp at once.
+    auto load_s = [&](uint32_t s, uint32_t (&sv)[64]) -> bool {
+      if (!ptx::mbar_wait(bar(bars->sfull[grp]), (s >> 1) & 1u, abort_flag)) return false;
       ptx::tc_fence_after();
-      ptx::tmem_ld32(tmem + lane_off + TM_S0 + sb * 128 + (uint32_t)col0, sv);
+      ptx::tmem_ld32(sbuf + lane_off + (uint32_t)col0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      ptx::tmem_ld32(sbuf + lane_off + (uint32_t)col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(bars->sfree[sb]));
-      ++scnt;
+      if (lane == 0) ptx::mbar_arrive(bar(bars->sfree[grp]));
       return true;
     };
-    // Column sums of this warp's 32 rows x 32 columns (after the recursive
-    // halving lane l holds column l), then across the four row quadrants in
-    // shared memory; the last of the four warps adds them to the global
-    // accumulator.  Integer sums do not depend on arrival order.
-    auto add_colsums = [&](const Item& t, int jt, float (&v)[32]) {
+    // Column sums of 32 rows x 32 columns held one row per lane: recursive
+    // halving (stages 0-4, run here from st0 to st1 - 1) leaves column `lane`
+    // in v[0].
+    auto warp_colsum = [&](float* v, int st0, int st1) -> float {
 #pragma unroll
-      for (int st = 0; st < 5; ++st) {
+      for (int st = st0; st < st1; ++st) {
         const int o = 16 >> st;
         const int hn = 16 >> st;
         const bool upper = (lane & o) != 0;
@@ -378,56 +405,44 @@ __global__ void __launch_bounds__(THREADS, 1)
           v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
         }
       }
-      const int par = jt & 1;
-      unsigned long long* acc = cs_acc + par * 128 + col0;
-      atomicAdd(&acc[lane], (unsigned long long)__double2ll_rn((double)v[0] * kImpScale));
-      __threadfence_block();
-      __syncwarp();
-      int last = 0;
-      if (lane == 0) last = atomicAdd(&cs_cnt[par * PARTS + part], 1) == 3;
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {
-        __threadfence_block();
-        const unsigned long long fx = atomicExch(&acc[lane], 0ull);
-        const int key = jt * KT + col0 + lane;
-        if (key < t.L && fx != 0ull) atomicAdd(&p.imp_acc[t.k0 + key], fx);
-        if (lane == 0) cs_cnt[par * PARTS + part] = 0;
-      }
+      return v[0];
     };
 
     for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
       const Item t = load_item(p, it);
-      uint32_t sv[32];
-      uint32_t sb, spar;
-      // ---- pass 1: max and normaliser of this warp's 32-column quarter
+      uint32_t sv[64];
+      // ---- pass 1: max and normaliser over this warp's tiles and column half
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < t.ntiles; ++j) {
-        if (!load_s(sv, sb, spar)) {
+        const uint32_t s = gs + (uint32_t)j;
+        if ((int)(s & 1u) != grp) continue;
+        if (!load_s(s, sv)) {
           failed = true;
           break;
         }
         const int kmax = t.L - j * KT - col0;  // columns >= kmax are outside the sequence
         if (kmax <= 0) continue;
-        float x[32];
+        float x[64];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(sv[c]);
-        if (kmax < 32) {
+        for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(sv[c]);
+        if (kmax < 64) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
+          for (int c = 0; c < 64; ++c)
             if (c >= kmax) x[c] = -INFINITY;
         }
         float mx[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-        for (int c = 4; c < 32; ++c) mx[c & 3] = fmaxf(mx[c & 3], x[c]);
+        for (int c = 4; c < 64; ++c) mx[c & 3] = fmaxf(mx[c & 3], x[c]);
         const float mn = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
         float sm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 32; ++c) sm[c & 3] += ex2(x[c] - mn);
-        l = l * ex2(m - mn) + ((sm[0] + sm[1]) + (sm[2] + sm[3]));
+        for (int c = 0; c < 64; ++c) sm[c & 3] += ex2(x[c] - mn);
+        l = (m == -INFINITY ? 0.f : l * ex2(m - mn)) + ((sm[0] + sm[1]) + (sm[2] + sm[3]));
         m = mn;
       }
       if (failed) break;
-      // merge the four quarters of every row once per item
+      gs += (uint32_t)t.ntiles;
+      // merge the four (group, half) parts of every row once per item
       float* st_par = stat + (ic & 1u) * (PARTS * 256);
       st_par[part * 256 + rl] = m;
       st_par[part * 256 + 128 + rl] = l;
@@ -450,50 +465,98 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float lse = rl < t.nrows ? M + __log2f(Ls) : INFINITY;
       // ---- pass 2: final probabilities -> P (TMEM, over its S tile); column sums
       for (int j = 0; j < t.ntiles; ++j) {
-        if (!load_s(sv, sb, spar)) {
-          failed = true;
-          break;
-        }
-        const int kmax = t.L - j * KT - col0;
-        float pv[32];
-        if (kmax >= 32) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pv[c] = ex2(__uint_as_float(sv[c]) - lse);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pv[c] = c < kmax ? ex2(__uint_as_float(sv[c]) - lse) : 0.f;
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(pv[2 * c], pv[2 * c + 1]);
-        // every quarter of the tile must have been read before P overwrites it
-        if (!ptx::mbar_wait(bar(bars->sfree[sb]), spar, abort_flag)) {
+        const uint32_t s = gs + (uint32_t)j;
+        if ((int)(s & 1u) != grp) continue;
+        const uint32_t scol = sbuf + lane_off + (uint32_t)col0;
+        const int kmax = t.L - j * KT - col0;  // columns >= kmax are outside the sequence
+        if (!ptx::mbar_wait(bar(bars->sfull[grp]), (s >> 1) & 1u, abort_flag)) {
           failed = true;
           break;
         }
         ptx::tc_fence_after();
-        ptx::tmem_st16(tmem + lane_off + TM_S0 + sb * 128 + (uint32_t)(col0 / 2), pk);
+        uint32_t* sa = &sv[0];
+        uint32_t* sb = &sv[32];
+        ptx::tmem_ld32(scol, *reinterpret_cast<uint32_t(*)[32]>(sa));
+        ptx::tmem_wait_ld();
+        // keys col0..col0+31 -> packed columns col0..col0+15 (already read)
+        float pv[32];
+        auto probs = [&](const uint32_t* x, int lim) {
+          if (lim >= 32) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) pv[c] = ex2(__uint_as_float(x[c]) - lse);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) pv[c] = c < lim ? ex2(__uint_as_float(x[c]) - lse) : 0.f;
+          }
+        };
+        auto store_p = [&](uint32_t col) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) pk[c] = pack_bf16(pv[2 * c], pv[2 * c + 1]);
+          ptx::tmem_st16(col, pk);
+        };
+        probs(sa, kmax);
+        store_p(scol);
+        // column sums of this warp's first 32 keys: the first halving step
+        // frees half of the registers, the rest overlaps the second load
+        if (p.want_imp) warp_colsum(pv, 0, 1);
+        ptx::tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(sb));
+        const int par = (int)((s >> 1) & 1u);
+        unsigned long long* cs_acc = cs_base + par * 128;
+        if (p.want_imp) {
+          const float c0 = warp_colsum(pv, 1, 5);
+          atomicAdd(&cs_acc[lane], (unsigned long long)__double2ll_rn((double)c0 * kImpScale));
+        }
+        ptx::tmem_wait_ld();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(bars->sfree[grp]));  // S tile fully read
+        // keys col0+32..col0+63 -> packed columns col0+16..col0+31
+        probs(sb, kmax - 32);
+        store_p(scol + 16);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(bars->pready));
-        if (p.want_imp) add_colsums(t, j, pv);
+        if (lane == 0) ptx::mbar_arrive(bar(bars->pready[grp]));
+        if (p.want_imp) {
+          const float c1 = warp_colsum(pv, 0, 5);
+          atomicAdd(&cs_acc[32 + lane], (unsigned long long)__double2ll_rn((double)c1 * kImpScale));
+          // the last of the four row quadrants adds the tile's sums to the keys
+          int* cs_cnt = cnt_base + par * 2;
+          __threadfence_block();
+          __syncwarp();
+          int last = 0;
+          if (lane == 0) last = atomicAdd(cs_cnt, 1) == 3;
+          last = __shfl_sync(0xffffffffu, last, 0);
+          if (last) {
+            __threadfence_block();
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const unsigned long long fx = atomicExch(&cs_acc[32 * e + lane], 0ull);
+              const int key = j * KT + col0 + 32 * e + lane;
+              if (key < t.L && fx != 0ull) atomicAdd(&p.imp_acc[t.k0 + key], fx);
+            }
+            if (lane == 0) *cs_cnt = 0;
+          }
+        }
       }
       if (failed) break;
-      // ---- O (already normalised) -> out
+      gs += (uint32_t)t.ntiles;
+      // ---- O (already normalised) -> out: warp sw takes columns 32*(sw/4)..+31
       if (!ptx::mbar_wait(bar(bars->ofull), ic & 1u, abort_flag)) {
         failed = true;
         break;
       }
       ptx::tc_fence_after();
-      ptx::tmem_ld32(tmem + lane_off + TM_O + (uint32_t)col0, sv);
+      const int ocol = 32 * (sw >> 2);
+      ptx::tmem_ld32(tmem + lane_off + TM_O + (uint32_t)ocol, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(bars->ofree));
       if (rl < t.nrows) {
         uint4* dst = reinterpret_cast<uint4*>(
-            p.out + ((size_t)(t.q0 + t.qt * QT + rl) * p.H + t.h) * HD + col0);
+            p.out + ((size_t)(t.q0 + t.qt * QT + rl) * p.H + t.h) * HD + ocol);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint4 w;
