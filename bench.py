@@ -34,6 +34,48 @@ METRIC = "query-tokens/s per fused Flash-Cache step (B=32, L=1536); % of rooflin
 UNIT = "query-tokens/s"
 
 
+# Sources whose SHA-256 (concatenated, first 16 hex digits) keys a committed
+# ncu traffic figure for each kernel.
+_KERNEL_SOURCES = {
+    "qkv_rope_scatter": ["qkv_tc.cu", "ptx.cuh", "fc_internal.h", "fc_api.cu"],
+    "attention": ["attn_tc.cu", "ptx.cuh", "fc_internal.h", "fc_api.cu"],
+}
+
+
+def _kernel_roofline(name, bound, work, timing, peaks, traffic):
+    """Achieved rate of one kernel (algorithmic work / mean launch time)."""
+    ms, n = timing
+    avg_s = ms / max(n, 1) / 1e3
+    if bound == "tensor":
+        achieved, peak, unit = work / avg_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    else:
+        achieved, peak, unit = work / avg_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+            "us_per_launch": avg_s * 1e6, "traffic": traffic}
+
+
+def _dram_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, for kernels whose
+    sources are unchanged since the capture (else absent -> null)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"dram_traffic_{workload}.txt")
+    out = {}
+    if not os.path.exists(path):
+        return out
+    csrc = os.path.join(ROOT, "kv_cache_attention_qkv_b200", "csrc")
+    for line in open(path):
+        f = line.split()
+        if not f or f[0].startswith("#") or len(f) < 5 or f[0] not in _KERNEL_SOURCES:
+            continue
+        h = hashlib.sha256()
+        for name in _KERNEL_SOURCES[f[0]]:
+            with open(os.path.join(csrc, name), "rb") as fh:
+                h.update(fh.read())
+        if f[1] == workload and h.hexdigest()[:16] == f[2]:
+            out[f[0]] = int(f[3]) + int(f[4])
+    return out
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -277,6 +319,7 @@ def run_ours(args):
             peak = peaks["hbm_gbs"]
             unit = "GB/s"
         t_roof = max(wk["flops"] / (peaks["bf16_tflops"] * 1e12), wk["bytes"] / (peaks["hbm_gbs"] * 1e9))
+        traffic = _dram_traffic(args.workload)
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -286,8 +329,10 @@ def run_ours(args):
                        "heads": H, "head_dim": d, "topk": K, "total_q": T, "total_k": S,
                        "l2": "flushed between steps (256 MiB write)", "parallelism": f"sequence-sharded x{ws}"},
             "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak, "traffic": traffic.get(dom),
                          "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst)"},
+            "kernel_rooflines": {k: _kernel_roofline(k, b, w, per_kernel[k], peaks, traffic.get(k))
+                                 for k, (b, w) in names.items()},
             "step_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": ms_per_step * 1e3,
                               "frac": t_roof / (ms_per_step / 1e3), "flops": wk["flops"], "bytes": wk["bytes"]},
             "kernels_ms_per_step": {k: v[0] / max(v[1], 1) for k, v in per_kernel.items()},
