@@ -167,6 +167,50 @@ FC_API fc_status fc_topk_tracked(fc_handle* h, void* stream, int batch, int tota
                           int32_t* tracked);
 
 /*
+ * fc_step_host — fc_step followed by fc_topk_tracked with the per-step inputs
+ * and outputs in host memory: the serving form of a step, in which the
+ * weights and the KV cache stay resident on the device, a step's query rows,
+ * positions and lengths come in and its attention output and tracked
+ * positions go out.
+ *   x, q_pos, cu_seqlens_q, cu_seqlens_k, total_q, total_k
+ *                 as for fc_step, but x, q_pos and both cu_seqlens in HOST
+ *                 memory.
+ *   k_cache, v_cache  dev, as for fc_step (updated in place).
+ *   cand_lo, cand_hi, k_per_seq (or NULL), k
+ *                 as for fc_topk_tracked, arrays in HOST memory.
+ *   out           HOST, [T, H, d] of dtype.
+ *   tracked       HOST, int32 [B, k] (may be NULL when k = 0).
+ * The importance of the step is computed into a handle-owned device buffer
+ * (fc_step gives access to it).
+ * The call returns once the work is queued; it does not wait for the GPU.
+ * Two handle-owned copy streams and two sets of device staging buffers let
+ * the input copy of one call and the output copy of the previous call run
+ * while the kernels of the current call run on `stream`.  Host input buffers
+ * must stay unchanged, and out / tracked must not be read, until the caller
+ * has called fc_host_sync(h, stream) and `stream` has reached that point
+ * (e.g. cudaStreamSynchronize).  Page-locked host memory makes the copies
+ * asynchronous; pageable memory is accepted but serialises the copies with
+ * the host.  The first call allocates the staging buffers (two copies of x,
+ * the small arrays, out and tracked, sized from the config) and the copy
+ * streams; FC_ERR_OOM / FC_ERR_CUDA if that fails.  Argument errors return
+ * FC_ERR_INVALID_ARG before anything is queued.  One handle: one stream.
+ */
+FC_API fc_status fc_step_host(fc_handle* h, void* stream, int batch, const void* x,
+                              const int32_t* q_pos, const int32_t* cu_seqlens_q,
+                              const int32_t* cu_seqlens_k, int total_q, int total_k,
+                              void* k_cache, void* v_cache, const int32_t* cand_lo,
+                              const int32_t* cand_hi, const int32_t* k_per_seq, int k, void* out,
+                              int32_t* tracked);
+
+/*
+ * fc_host_sync — make `stream` wait (on the device, without blocking the
+ * host) until every copy queued by earlier fc_step_host calls has completed.
+ * After cudaStreamSynchronize(stream) the host outputs of all those calls are
+ * complete and their host inputs are no longer read.
+ */
+FC_API fc_status fc_host_sync(fc_handle* h, void* stream);
+
+/*
  * fc_get_error — wait for the stream of the handle's last call, copy the
  * device error word to *device_error_word (host) and clear it.
  * Returns FC_OK when the word was 0, FC_ERR_TIMEOUT when it holds

@@ -22,9 +22,9 @@ FC_DTYPE_FP32 = 1
 STATUS = {0: "FC_OK", -1: "FC_ERR_INVALID_ARG", -2: "FC_ERR_UNSUPPORTED", -3: "FC_ERR_CUDA",
           -4: "FC_ERR_OOM", -5: "FC_ERR_DEVICE_CHECK", -6: "FC_ERR_TIMEOUT"}
 DEVERR = {0x01: "POS_RANGE", 0x02: "POS_DUP", 0x04: "SEQLENS", 0x08: "CAND", 0x10: "TIMEOUT"}
-EXPORTED = ("fc_create", "fc_step", "fc_topk_tracked", "fc_get_error", "fc_last_launch_count",
-            "fc_profile", "fc_profile_read", "fc_attention_noalloc", "fc_selftest_wait_timeout",
-            "fc_destroy", "fc_status_str")
+EXPORTED = ("fc_create", "fc_step", "fc_topk_tracked", "fc_step_host", "fc_host_sync",
+            "fc_get_error", "fc_last_launch_count", "fc_profile", "fc_profile_read",
+            "fc_attention_noalloc", "fc_selftest_wait_timeout", "fc_destroy", "fc_status_str")
 PROFILE_SLOTS = ("prep", "qkv_rope_scatter", "attention", "importance_finalize", "topk")
 
 
@@ -61,6 +61,11 @@ def load_library(path: Optional[str] = None):
     lib.fc_step.restype = c_int
     lib.fc_topk_tracked.argtypes = [vp, vp, c_int, c_int, vp, vp, vp, vp, vp, c_int, vp]
     lib.fc_topk_tracked.restype = c_int
+    lib.fc_step_host.argtypes = [vp, vp, c_int, vp, vp, vp, vp, c_int, c_int, vp, vp, vp, vp, vp,
+                                 c_int, vp, vp]
+    lib.fc_step_host.restype = c_int
+    lib.fc_host_sync.argtypes = [vp, vp]
+    lib.fc_host_sync.restype = c_int
     lib.fc_get_error.argtypes = [vp, i32p]
     lib.fc_get_error.restype = c_int
     lib.fc_last_launch_count.argtypes = [vp]
@@ -173,6 +178,44 @@ class FlashCache:
                                       _ptr(cand_hi), _ptr(k_per_seq), int(k), _ptr(tracked))
         if st != 0:
             raise FlashCacheError(st, "fc_topk_tracked")
+
+    def _check_host(self, t: torch.Tensor, name: str, dtype, ndim: int):
+        if t.dtype != dtype or t.is_cuda or not t.is_contiguous() or t.dim() != ndim:
+            raise FlashCacheError(-1, f"{name}: need a contiguous {dtype} host tensor, {ndim}-D")
+
+    def step_host(self, x, q_pos, cu_seqlens_q, cu_seqlens_k, k_cache, v_cache, cand_lo, cand_hi,
+                  k: int, out, tracked, k_per_seq=None, stream=None) -> None:
+        """Enqueue fc_step_host: host (ideally pinned) inputs and outputs, device
+        KV cache.  Outputs are valid after host_sync() and a sync of ``stream``."""
+        H, d = self.n_heads, self.head_dim
+        self._check_host(x, "x", self.dtype, 2)
+        for n, t in (("q_pos", q_pos), ("cu_seqlens_q", cu_seqlens_q),
+                     ("cu_seqlens_k", cu_seqlens_k), ("cand_lo", cand_lo), ("cand_hi", cand_hi)):
+            self._check_host(t, n, torch.int32, 1)
+        if k_per_seq is not None:
+            self._check_host(k_per_seq, "k_per_seq", torch.int32, 1)
+        self._check_host(out, "out", self.dtype, 3)
+        self._check_host(tracked, "tracked", torch.int32, 2)
+        for n, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+            self._check(t, n, self.dtype, 3)
+        T, S = x.shape[0], k_cache.shape[0]
+        B = cu_seqlens_q.shape[0] - 1
+        if (x.shape[1] != self.hidden or q_pos.shape[0] != T or tuple(out.shape) != (T, H, d)
+                or v_cache.shape[0] != S or cu_seqlens_k.shape[0] != B + 1
+                or tuple(tracked.shape) != (B, k) or cand_lo.shape[0] != B or cand_hi.shape[0] != B):
+            raise FlashCacheError(-1, "fc_step_host: inconsistent shapes")
+        st = self.lib.fc_step_host(self._h, _stream_handle(stream), B, _ptr(x), _ptr(q_pos),
+                                   _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), T, S, _ptr(k_cache),
+                                   _ptr(v_cache), _ptr(cand_lo), _ptr(cand_hi), _ptr(k_per_seq),
+                                   int(k), _ptr(out), _ptr(tracked))
+        if st != 0:
+            raise FlashCacheError(st, "fc_step_host")
+
+    def host_sync(self, stream=None) -> None:
+        """Make ``stream`` wait for every copy queued by step_host (fc_host_sync)."""
+        st = self.lib.fc_host_sync(self._h, _stream_handle(stream))
+        if st != 0:
+            raise FlashCacheError(st, "fc_host_sync")
 
     def get_error(self) -> int:
         """Wait for the last stream used and return (and clear) the device error word."""

@@ -393,6 +393,7 @@ void fc_destroy(fc_handle* h) {
   cudaSetDevice(h->device);
   cudaDeviceSynchronize();
   free_workspace(h);
+  fc::free_host_pipe(h);
   if (h->prof_ev) {
     for (int i = 0; i < 2 * 4096; ++i) cudaEventDestroy(h->prof_ev[i]);
     delete[] h->prof_ev;

@@ -53,6 +53,21 @@ struct StepShape {
 
 }  // namespace fc
 
+namespace fc {
+// Device staging and copy streams of fc_step_host (allocated on first use).
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t s_h2d = nullptr, s_d2h = nullptr;
+  void* x[2] = {nullptr, nullptr};        // [max_total_q, hidden] dtype
+  int32_t* small[2] = {nullptr, nullptr}; // q_pos | cu_q | cu_k | lo | hi | k_per_seq
+  void* out[2] = {nullptr, nullptr};      // [max_total_q, H, d] dtype
+  int32_t* tracked[2] = {nullptr, nullptr};  // [max_batch, max_topk]
+  float* importance = nullptr;            // [max_total_k]
+  cudaEvent_t h2d_done[2] = {}, comp_done[2] = {}, d2h_done[2] = {};
+  unsigned long long calls = 0;
+};
+}  // namespace fc
+
 struct fc_handle {
   fc_config cfg;
   int device = 0;
@@ -71,7 +86,12 @@ struct fc_handle {
   cudaEvent_t* prof_ev = nullptr;  // 2 * 4096 events, created on first fc_profile(1)
   CUtensorMap tm_w;  // W_qkv, bf16 tensor-core path
   CUtensorMap tm_q;  // Q buffer, bf16 tensor-core path
+  fc::HostPipe hp;   // fc_step_host
 };
+
+namespace fc {
+void free_host_pipe(fc_handle* h);
+}
 
 namespace fc {
 

@@ -209,3 +209,52 @@ def test_bounded_wait_times_out_and_context_stays_usable():
     gpu = tl.run_gpu(inp, layer=layer, dev=dev)
     assert gpu["err"] == 0
     tl.compare_step(inp, gpu, tl.run_oracle(inp), range(inp.batch))
+
+
+@pytest.mark.parametrize("name", ["small_varlen", "tiny_fp32"])
+def test_step_host_matches_device_path(name):
+    """fc_step_host (host inputs and outputs, copies double-buffered against the
+    kernels) gives the same bits as fc_step + fc_topk_tracked on device buffers,
+    over consecutive calls with different inputs: both staging sets, then their
+    reuse."""
+    inp = workloads.generate(name)
+    dev_a, dev_b = tl.upload(inp), tl.upload(inp)
+    layer_a, layer_b = tl.make_layer(inp, dev_a["w"]), tl.make_layer(inp, dev_b["w"])
+    T, S, H, d, B = inp.total_q, inp.total_k, inp.n_heads, inp.head_dim, inp.batch
+    K = int(inp.topk.max())
+    dt = dev_a["x"].dtype
+    scales = (1.0, -0.5, 0.25, 2.0)
+    want_out, want_tr = [], []
+    for sc in scales:
+        out = torch.empty((T, H, d), device="cuda", dtype=dt)
+        imp = torch.empty((S,), device="cuda")
+        tr = torch.empty((B, K), device="cuda", dtype=torch.int32)
+        layer_a.step(dev_a["x"] * sc, dev_a["q_pos"], dev_a["cu_q"], dev_a["cu_k"],
+                     dev_a["k_cache"], dev_a["v_cache"], out, imp)
+        layer_a.topk_tracked(imp, dev_a["cu_k"], dev_a["cand_lo"], dev_a["cand_hi"], K, tr,
+                             k_per_seq=dev_a["topk"])
+        want_out.append(out.cpu())
+        want_tr.append(tr.cpu())
+    assert layer_a.get_error() == 0
+
+    pin = lambda t: t.cpu().contiguous().pin_memory()
+    xs = [pin(dev_b["x"] * sc) for sc in scales]
+    small = {n: pin(dev_b[n]) for n in ("q_pos", "cu_q", "cu_k", "cand_lo", "cand_hi", "topk")}
+    outs = [torch.full((T, H, d), float("nan"), dtype=dt).pin_memory() for _ in scales]
+    trs = [torch.full((B, K), -7, dtype=torch.int32).pin_memory() for _ in scales]
+    torch.cuda.synchronize()
+    for i in range(len(scales)):
+        layer_b.step_host(xs[i], small["q_pos"], small["cu_q"], small["cu_k"], dev_b["k_cache"],
+                          dev_b["v_cache"], small["cand_lo"], small["cand_hi"], K, outs[i], trs[i],
+                          k_per_seq=small["topk"])
+    layer_b.host_sync()
+    torch.cuda.synchronize()
+    assert layer_b.get_error() == 0
+    bits = torch.int16 if dt == torch.bfloat16 else torch.int32
+    for i in range(len(scales)):
+        assert torch.equal(outs[i].view(bits), want_out[i].view(bits)), f"out of call {i}"
+        assert torch.equal(trs[i], want_tr[i]), f"tracked of call {i}"
+    for n in ("k_cache", "v_cache"):
+        assert torch.equal(dev_b[n].view(bits), dev_a[n].view(bits)), n
+    layer_a.close()
+    layer_b.close()
