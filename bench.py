@@ -190,7 +190,8 @@ def run_ours(args):
     dev = torch.device("cuda", torch.cuda.current_device())
 
     # every rank draws its own batch of the same recipe
-    inp = workloads.generate(args.workload, seed=workloads.WORKLOADS.index(args.workload) + 1000 * rank)
+    base_seed = workloads.WORKLOADS.index(args.workload) if args.workload in workloads.WORKLOADS else 100
+    inp = workloads.generate(args.workload, seed=base_seed + 1000 * rank)
     dt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
     f = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dtype=dt)
     i = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
@@ -420,6 +421,16 @@ def run_reference(args):
     }
 
 
+# Sweep axes (the pages' measured axes, throughput side): batch size at the
+# headline query and cache, query size beta_m at batch 32, cache length at
+# batch 32 and beta_m 128.
+SWEEPS = {
+    "batch": [f"sweep_b{b}_m128_L1536" for b in (1, 2, 4, 8, 16, 32, 64)],
+    "beta": [f"sweep_b32_m{m}_L1536" for m in (64, 128, 192, 256)],
+    "cache": [f"sweep_b32_m128_L{L}" for L in (768, 1536, 3072, 4096, 8192)],
+}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -429,9 +440,23 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of oracle time for cpu_baseline (0 = skip)")
+    ap.add_argument("--sweep", choices=sorted(SWEEPS) + ["all"], default=None,
+                    help="time every point of a sweep axis (one JSON line per point, no cpu_baseline)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.sweep is not None:
+        if args.impl != "ours":
+            ap.error("--sweep times this implementation only")
+        axes = sorted(SWEEPS) if args.sweep == "all" else [args.sweep]
+        for axis in axes:
+            for point in SWEEPS[axis]:
+                args.workload, args.cpu_budget = point, 0.0
+                res = run_ours(args)
+                if res is not None:
+                    res["sweep"] = axis
+                    print(json.dumps(res), flush=True)
+        return
     res = run_reference(args) if args.impl == "reference" else run_ours(args)
     if res is not None:
         print(json.dumps(res), flush=True)

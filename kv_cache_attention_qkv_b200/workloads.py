@@ -18,6 +18,12 @@ Five workloads are defined, named by what they are:
 * ``small_d64``      bf16 with head_dim 64 (the CUDA-core path): B=2, hidden
                      96, 3 heads x 64, caches of 200 and 333 rows.
 
+Sweep points are named ``sweep_b<B>_m<beta>_L<L>``: the headline recipe with
+B sequences, a query of beta rows (beta/2 tracked + a beta/2-row window) and a
+cache of L rows per sequence (the generated span is the last 512 rows, or the
+last half of the cache when it is shorter).  They mirror the axes the pages
+measure (batch size, query size beta_m, cache length).
+
 The shapes follow LLaDA-8B (the model the Flash-dLLM pages evaluate); weights
 and caches are random, there is no dataset and no checkpoint.
 
@@ -114,19 +120,44 @@ def _layout(rng, lens_k: List[int], windows: List[int], budgets: List[int],
     return np.concatenate(pos_rows).astype(np.int32), cu_q, cu_k
 
 
+def parse_sweep(name: str):
+    """(B, beta, L) of a ``sweep_b<B>_m<beta>_L<L>`` name, else None."""
+    import re
+
+    m = re.fullmatch(r"sweep_b(\d+)_m(\d+)_L(\d+)", name)
+    if not m:
+        return None
+    B, beta, L = (int(v) for v in m.groups())
+    if B < 1 or beta < 2 or beta % 2 or L < 2 * beta:
+        raise ValueError(f"bad sweep point {name!r}: need B >= 1, even beta >= 2, L >= 2 beta")
+    return B, beta, L
+
+
 def generate(name: str, seed: Optional[int] = None, batch: Optional[int] = None) -> StepInputs:
     """Draw the named workload.  ``seed`` defaults to the workload's index.
 
     ``batch`` overrides the number of sequences (used to draw a sub-sample or a
     per-rank shard of the same recipe); per-sequence draws keep their recipe.
     """
-    if name not in WORKLOADS:
-        raise ValueError(f"unknown workload {name!r}; known: {WORKLOADS}")
+    sweep = parse_sweep(name)
+    if name not in WORKLOADS and sweep is None:
+        raise ValueError(f"unknown workload {name!r}; known: {WORKLOADS} and sweep_b<B>_m<beta>_L<L>")
     if seed is None:
-        seed = WORKLOADS.index(name)
+        seed = WORKLOADS.index(name) if sweep is None else 100
     rng = np.random.default_rng(seed)
 
-    if name == "tiny_fp32":
+    if sweep is not None:
+        dtype, D, H, d, theta, w_std = "bf16", 4096, 32, 128, 5.0e5, 0.02
+        B0, beta, L = sweep
+        B = batch or B0
+        half = beta // 2
+        gen = min(512, L // 2)  # generated span: the last `gen` rows of the cache
+        lens = [L] * B
+        windows = [half] * B
+        budgets = [half] * B
+        n_slots = (gen - half) // half + 1
+        starts = [int(L - gen + half * rng.integers(0, n_slots)) for _ in range(B)]
+    elif name == "tiny_fp32":
         dtype, D, H, d, theta, w_std = "fp32", 32, 2, 16, 1.0e4, 0.1
         B = batch or 1
         lens = [64] * B

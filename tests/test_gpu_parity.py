@@ -30,7 +30,11 @@ def test_full_parity(name):
 
 @pytest.mark.slow
 @pytest.mark.parametrize("name,seqs", [("batch32_uniform", [0, 13, 31]),
-                                       ("batch32_varlen", [0, 5, 17, 30])])
+                                       ("batch32_varlen", [0, 5, 17, 30]),
+                                       # sweep extremes: two 128-row query tiles per
+                                       # sequence over an 8192-row cache; 64 sequences
+                                       ("sweep_b2_m256_L8192", [0, 1]),
+                                       ("sweep_b64_m128_L1536", [0, 40, 63])])
 def test_full_size_sampled_parity(name, seqs):
     """Full-size workloads, same launch configuration as the bench; the oracle
     recomputes sampled sequences (sequences are independent)."""

@@ -344,3 +344,23 @@ def test_varlen_workload_recipe():
     assert (inp.window_start % inp.window_len == 0).all()
     assert (inp.window_start >= L - 512).all()
     assert (inp.window_start + inp.window_len <= L).all()
+
+
+@pytest.mark.parametrize("name,B,beta,L", [("sweep_b1_m64_L768", 1, 64, 768),
+                                           ("sweep_b3_m256_L600", 3, 256, 600)])
+def test_sweep_workload_recipe(name, B, beta, L):
+    """Sweep points: B sequences of L cache rows, beta/2 tracked + beta/2 window rows,
+    the window inside the generated span (the last min(512, L/2) rows)."""
+    assert workloads.parse_sweep(name) == (B, beta, L)
+    inp = workloads.generate(name)
+    assert inp.batch == B and (np.diff(inp.cu_seqlens_k) == L).all()
+    assert (np.diff(inp.cu_seqlens_q) == beta).all()
+    assert (inp.window_len == beta // 2).all() and (inp.topk == beta // 2).all()
+    gen = min(512, L // 2)
+    assert (inp.window_start >= L - gen).all() and (inp.window_start + beta // 2 <= L).all()
+    for b in range(B):
+        pos = inp.q_pos[inp.seq_slice_q(b)]
+        assert len(np.unique(pos)) == beta and (pos[: beta // 2] < inp.window_start[b]).all()
+    with pytest.raises(ValueError):
+        workloads.parse_sweep("sweep_b1_m63_L768")
+    assert workloads.parse_sweep("batch32_uniform") is None
