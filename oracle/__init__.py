@@ -1,4 +1,5 @@
-"""Plain fp64 CPU oracle of one Flash-Cache step (test infrastructure only).
+"""Plain fp64 CPU oracle of one Flash-Cache step and of the model step around
+it (``model_oracle``); test infrastructure only.
 
 Only the tests, the package's ``__graft_entry__.smoke()`` check and the CPU
 baseline leg of ``bench.py`` may import this package.  The CUDA library never
@@ -16,3 +17,4 @@ from .flashcache_oracle import (  # noqa: F401
     flashcache_step,
     topk_tracked,
 )
+from . import model_oracle  # noqa: F401,E402
