@@ -284,6 +284,97 @@ FC_API fc_status fc_attention_noalloc(void* stream, int dtype, int batch, int n_
  * on the handle's device first (cudaDeviceSynchronize). */
 FC_API void fc_destroy(fc_handle* h);
 
+/* ==========================================================================
+ * Model step: the decoder stack around the Flash-Cache layer.
+ *
+ * The Flash-dLLM pages evaluate LLaDA-8B (paper-digest page, evaluation;
+ * forum post, configuration table).  One model step runs the query rows of
+ * every sequence (tracked positions + masked window) through n_layers
+ * LLaMA-style decoder layers, each attending through the Flash-Cache step of
+ * fc_step (its own K/V cache per layer), then scores the rows the caller names
+ * with the LM head: per row the top token, its softmax probability (the
+ * confidence) and the Flash-Verify acceptance confidence >= threshold
+ * (paper-digest page, Flash-Verify; threshold 0.9 in the configuration).
+ * Layer (no biases; rms_norm(x) = x / sqrt(mean(x^2) + eps)):
+ *   h += Wo . attn(rms_norm(h) * g_attn)
+ *   h += Wd . (silu(Wg . m) * (Wu . m)),  m = rms_norm(h) * g_mlp
+ * and the LM head reads rms_norm(h) * g_final.  Every activation between
+ * kernels is bf16; each kernel accumulates in fp32.
+ * ========================================================================== */
+typedef struct fc_model_config {
+  fc_config layer;      /* attention layer: dtype FC_DTYPE_BF16, head_dim 128,
+                           n_heads even, hidden a multiple of 256; the max_*
+                           limits bound every step as for fc_create */
+  int n_layers;         /* >= 1 */
+  int intermediate;     /* SwiGLU width I, a multiple of 128 */
+  int vocab;            /* V >= 1 */
+  int max_head_rows;    /* rows the LM head may score per step, >= 1 */
+  float rms_eps;        /* e.g. 1e-5 */
+  float threshold;      /* acceptance threshold on the confidence, e.g. 0.9 */
+} fc_model_config;
+
+/* One decoder layer's weights: device pointers, bf16, row-major, 16-byte
+ * aligned, kept by pointer until fc_model_destroy. */
+typedef struct fc_layer_weights {
+  const void* attn_norm;  /* [D] */
+  const void* w_qkv;      /* [3*H*d, D], as for fc_create */
+  const void* w_o;        /* [D, H*d] */
+  const void* mlp_norm;   /* [D] */
+  const void* w_gate;     /* [I, D] */
+  const void* w_up;       /* [I, D] */
+  const void* w_down;     /* [D, I] */
+} fc_layer_weights;
+
+typedef struct fc_model fc_model;
+
+/*
+ * fc_model_create — validate `cfg`, bind the weights (`layers`: host array of
+ * n_layers entries; final_norm dev [D]; lm_head dev [V, D]) and allocate the
+ * workspace (one Flash-Cache handle for the attention of every layer, the
+ * bf16 activations h, a [max_total_q, D], o [max_total_q, H*d],
+ * s [max_total_q, I], the LM-head rows [max_head_rows, D] and statistics).
+ * FC_ERR_UNSUPPORTED for shapes outside the tensor-core path,
+ * FC_ERR_INVALID_ARG for NULL or misaligned pointers, FC_ERR_OOM / FC_ERR_CUDA.
+ */
+FC_API fc_status fc_model_create(const fc_model_config* cfg, const fc_layer_weights* layers,
+                                 const void* final_norm, const void* lm_head, fc_model** out);
+
+/*
+ * fc_model_step — one model step on a packed, variable-length batch.
+ *   batch, q_pos, cu_seqlens_q, cu_seqlens_k, total_q (>= 1), total_k
+ *                 as for fc_step (dev).
+ *   x             dev, [T, D] bf16: the input embeddings of the query rows.
+ *   k_caches, v_caches  host arrays of n_layers dev pointers, [S, H, d] bf16
+ *                 each, updated in place as by fc_step for every layer.
+ *   head_rows     dev, int32 [n_head_rows]: packed query rows (0 <= r < T) the
+ *                 LM head scores; n_head_rows 0 skips the head.
+ *   importance    dev, float [S] or NULL: the attention importance summed over
+ *                 every layer (overwritten).
+ *   token         dev, int32 [n_head_rows]: index of the largest logit (the
+ *                 lowest index on ties).
+ *   confidence    dev, float [n_head_rows]: its softmax probability.
+ *   accept        dev, uint8 [n_head_rows]: confidence >= threshold.
+ *   h_out         dev, [T, D] bf16 or NULL: the residual stream after the
+ *                 last layer.
+ * Enqueued on `stream`; device-side checks and timeouts go to the error word
+ * of the model's layer handle (fc_model_layer_handle + fc_get_error).
+ */
+FC_API fc_status fc_model_step(fc_model* m, void* stream, int batch, const void* x,
+                               const int32_t* q_pos, const int32_t* cu_seqlens_q,
+                               const int32_t* cu_seqlens_k, int total_q, int total_k,
+                               void* const* k_caches, void* const* v_caches,
+                               const int32_t* head_rows, int n_head_rows, float* importance,
+                               int32_t* token, float* confidence, uint8_t* accept, void* h_out);
+
+/* The Flash-Cache handle the model runs its attention through (owned by the
+ * model): for fc_topk_tracked on the model's importance, fc_get_error,
+ * fc_profile and fc_last_launch_count (which then counts the model step's
+ * kernels). */
+FC_API fc_handle* fc_model_layer_handle(fc_model* m);
+
+/* Release the model, its layer handle and workspace (NULL is a no-op). */
+FC_API void fc_model_destroy(fc_model* m);
+
 /* Static, human-readable name of a status. */
 FC_API const char* fc_status_str(fc_status s);
 

@@ -9,7 +9,7 @@ library has not been built: there is no fallback.
 """
 import importlib
 
-__all__ = ["FlashCache", "FlashCacheError", "load_library"]
+__all__ = ["FlashCache", "FlashCacheModel", "FlashCacheError", "load_library"]
 
 
 def __getattr__(name):

@@ -24,7 +24,8 @@ STATUS = {0: "FC_OK", -1: "FC_ERR_INVALID_ARG", -2: "FC_ERR_UNSUPPORTED", -3: "F
 DEVERR = {0x01: "POS_RANGE", 0x02: "POS_DUP", 0x04: "SEQLENS", 0x08: "CAND", 0x10: "TIMEOUT"}
 EXPORTED = ("fc_create", "fc_step", "fc_topk_tracked", "fc_step_host", "fc_host_sync",
             "fc_get_error", "fc_last_launch_count", "fc_profile", "fc_profile_read",
-            "fc_attention_noalloc", "fc_selftest_wait_timeout", "fc_destroy", "fc_status_str")
+            "fc_attention_noalloc", "fc_selftest_wait_timeout", "fc_destroy", "fc_status_str",
+            "fc_model_create", "fc_model_step", "fc_model_layer_handle", "fc_model_destroy")
 PROFILE_SLOTS = ("prep", "qkv_rope_scatter", "attention", "importance_finalize", "topk")
 
 
@@ -41,6 +42,19 @@ class FcConfig(ctypes.Structure):
                 ("max_total_k", ctypes.c_int), ("max_seqlen_q", ctypes.c_int),
                 ("max_pos", ctypes.c_int), ("max_topk", ctypes.c_int)]
 
+
+class FcModelConfig(ctypes.Structure):
+    _fields_ = [("layer", FcConfig), ("n_layers", ctypes.c_int), ("intermediate", ctypes.c_int),
+                ("vocab", ctypes.c_int), ("max_head_rows", ctypes.c_int),
+                ("rms_eps", ctypes.c_float), ("threshold", ctypes.c_float)]
+
+
+class FcLayerWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("attn_norm", "w_qkv", "w_o", "mlp_norm", "w_gate", "w_up", "w_down")]
+
+
+LAYER_WEIGHT_NAMES = tuple(n for n, _ in FcLayerWeights._fields_)
 
 _lib = None
 
@@ -81,6 +95,16 @@ def load_library(path: Optional[str] = None):
     lib.fc_attention_noalloc.restype = c_int
     lib.fc_destroy.argtypes = [vp]
     lib.fc_destroy.restype = None
+    lib.fc_model_create.argtypes = [ctypes.POINTER(FcModelConfig), ctypes.POINTER(FcLayerWeights),
+                                    vp, vp, ctypes.POINTER(vp)]
+    lib.fc_model_create.restype = c_int
+    lib.fc_model_step.argtypes = [vp, vp, c_int, vp, vp, vp, vp, c_int, c_int, vp, vp, vp, c_int,
+                                  vp, vp, vp, vp, vp]
+    lib.fc_model_step.restype = c_int
+    lib.fc_model_layer_handle.argtypes = [vp]
+    lib.fc_model_layer_handle.restype = vp
+    lib.fc_model_destroy.argtypes = [vp]
+    lib.fc_model_destroy.restype = None
     lib.fc_status_str.argtypes = [c_int]
     lib.fc_status_str.restype = ctypes.c_char_p
     if path is None:
@@ -270,3 +294,79 @@ class FlashCache:
 
 def describe_error_word(word: int):
     return [name for bit, name in DEVERR.items() if word & bit]
+
+
+class FlashCacheModel:
+    """The decoder stack around the Flash-Cache layer (fc_model_* of the C ABI):
+    weights bound at construction, model steps on demand."""
+
+    def __init__(self, layers, final_norm: torch.Tensor, lm_head: torch.Tensor, *, hidden: int,
+                 n_heads: int, head_dim: int, rope_theta: float, intermediate: int, max_batch: int,
+                 max_total_q: int, max_total_k: int, max_seqlen_q: int, max_pos: int,
+                 max_topk: int, max_head_rows: int, rms_eps: float = 1e-5,
+                 threshold: float = 0.9):
+        self.lib = load_library()
+        for t in [final_norm, lm_head] + [lw[n] for lw in layers for n in LAYER_WEIGHT_NAMES]:
+            if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+                raise FlashCacheError(-1, "model weights must be contiguous bfloat16 CUDA tensors")
+        self._keep = (layers, final_norm, lm_head)  # the library keeps the pointers
+        self.n_layers, self.hidden = len(layers), hidden
+        self.n_heads, self.head_dim = n_heads, head_dim
+        self.device = lm_head.device
+        cfg = FcModelConfig(FcConfig(hidden, n_heads, head_dim, float(rope_theta), FC_DTYPE_BF16,
+                                     max_batch, max_total_q, max_total_k, max_seqlen_q, max_pos,
+                                     max_topk),
+                            len(layers), intermediate, lm_head.shape[0], max_head_rows,
+                            float(rms_eps), float(threshold))
+        arr = (FcLayerWeights * len(layers))()
+        for i, lw in enumerate(layers):
+            for n in LAYER_WEIGHT_NAMES:
+                setattr(arr[i], n, lw[n].data_ptr())
+        h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            st = self.lib.fc_model_create(ctypes.byref(cfg), arr, _ptr(final_norm), _ptr(lm_head),
+                                          ctypes.byref(h))
+        if st != 0:
+            raise FlashCacheError(st, "fc_model_create")
+        self._m = h
+
+    def step(self, x, q_pos, cu_seqlens_q, cu_seqlens_k, k_caches, v_caches, head_rows=None,
+             importance=None, token=None, confidence=None, accept=None, h_out=None,
+             stream=None) -> None:
+        """Enqueue fc_model_step; k_caches / v_caches are lists of [S, H, d] tensors."""
+        if len(k_caches) != self.n_layers or len(v_caches) != self.n_layers:
+            raise FlashCacheError(-1, "one K and one V cache per layer")
+        T, S = x.shape[0], k_caches[0].shape[0]
+        B = cu_seqlens_q.shape[0] - 1
+        kp = (ctypes.c_void_p * self.n_layers)(*[t.data_ptr() for t in k_caches])
+        vp_ = (ctypes.c_void_p * self.n_layers)(*[t.data_ptr() for t in v_caches])
+        R = 0 if head_rows is None else head_rows.shape[0]
+        st = self.lib.fc_model_step(self._m, _stream_handle(stream), B, _ptr(x), _ptr(q_pos),
+                                    _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), T, S, kp, vp_,
+                                    _ptr(head_rows), R, _ptr(importance), _ptr(token),
+                                    _ptr(confidence), _ptr(accept), _ptr(h_out))
+        if st != 0:
+            raise FlashCacheError(st, "fc_model_step")
+
+    def get_error(self) -> int:
+        """Wait for the last stream used and return (and clear) the device error word."""
+        w = ctypes.c_int32(0)
+        st = self.lib.fc_get_error(self.lib.fc_model_layer_handle(self._m), ctypes.byref(w))
+        if st not in (0, -5, -6):
+            raise FlashCacheError(st, "fc_get_error")
+        return int(w.value)
+
+    @property
+    def last_launch_count(self) -> int:
+        return int(self.lib.fc_last_launch_count(self.lib.fc_model_layer_handle(self._m)))
+
+    def close(self) -> None:
+        if getattr(self, "_m", None):
+            self.lib.fc_model_destroy(self._m)
+            self._m = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

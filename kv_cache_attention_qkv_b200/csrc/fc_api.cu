@@ -233,6 +233,17 @@ fc_status fc_step(fc_handle* h, void* stream, int batch, const void* x, const in
                   int total_k, void* k_cache, void* v_cache, void* out, float* importance,
                   int accumulate) {
   if (!h) return FC_ERR_INVALID_ARG;
+  return fc::step_impl(h, &h->tm_w, stream, batch, x, q_pos, cu_seqlens_q, cu_seqlens_k, total_q,
+                       total_k, k_cache, v_cache, out, importance, accumulate);
+}
+
+}  // extern "C"
+
+fc_status fc::step_impl(fc_handle* h, const CUtensorMap* tm_w, void* stream, int batch,
+                        const void* x, const int32_t* q_pos,
+                        const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int total_q,
+                        int total_k, void* k_cache, void* v_cache, void* out, float* importance,
+                        int accumulate) {
   const fc_config& c = h->cfg;
   if (batch < 1 || batch > c.max_batch || total_q < 0 || total_q > c.max_total_q || total_k < 0 ||
       total_k > c.max_total_k || (accumulate != 0 && accumulate != 1))
@@ -271,7 +282,7 @@ fc_status fc_step(fc_handle* h, void* stream, int batch, const void* x, const in
                             (uint64_t)c.hidden * 2, fc::kQkvXBoxRows, 64))
       return FC_ERR_CUDA;
     ProfScope ps(h, st, 1);
-    e = fc::launch_qkv_tc(h, st, s, tm_x, q_pos, k_cache, v_cache);
+    e = fc::launch_qkv_tc(h, st, s, tm_x, *tm_w, q_pos, k_cache, v_cache);
   } else {
     ProfScope ps(h, st, 1);
     e = fc::launch_qkv_simt(h, st, s, x, q_pos, k_cache, v_cache);
@@ -302,6 +313,8 @@ fc_status fc_step(fc_handle* h, void* stream, int batch, const void* x, const in
   }
   return FC_OK;
 }
+
+extern "C" {
 
 fc_status fc_topk_tracked(fc_handle* h, void* stream, int batch, int total_k,
                           const float* importance, const int32_t* cu_seqlens_k,

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -19,6 +20,23 @@ constexpr int kSimtQTile = 16;
 // of a pair loads 128 rows of X and 128 rows (half the 256-row tile) of W.
 constexpr int kQkvXBoxRows = 128;
 constexpr int kQkvWBoxRows = 128;
+// TMA boxes of the model's other projections (gemm_tc): 128 rows x 64 columns
+// for both operands.
+constexpr int kGemmBoxRows = 128;
+
+// Epilogues of the generic tensor-core GEMM (gemm_tc.cu).
+enum GemmMode { GEMM_RESID = 0, GEMM_SWIGLU = 1, GEMM_LMHEAD = 2 };
+
+struct GemmParams {
+  int mode;
+  int M, N, K;     // rows of A, output columns (SwiGLU: features), reduction length
+  int num_m, num_n, num_tiles, num_k;  // filled by the launcher
+  const __nv_bfloat16* resid;  // GEMM_RESID: [M, ldo] added to the product (may equal out)
+  __nv_bfloat16* out;          // GEMM_RESID / GEMM_SWIGLU: [M, ldo]
+  size_t ldo;                  // row stride of resid / out in elements
+  float* partials;             // GEMM_LMHEAD: [M, num_n, 3] (max, sum exp, argmax bits)
+  int32_t* err;
+};
 
 // Importance is accumulated in fixed point (int64, 2^-40 units) so that the
 // sum over heads and query tiles is exact and independent of the order in
@@ -124,8 +142,22 @@ cudaError_t launch_attn_simt(const fc_handle* h, cudaStream_t st, const StepShap
                              const int32_t* cu_q, const int32_t* cu_k, const void* k_cache,
                              const void* v_cache, void* out, bool want_importance);
 cudaError_t launch_qkv_tc(const fc_handle* h, cudaStream_t st, const StepShape& s,
-                          const CUtensorMap& tm_x, const int32_t* q_pos, void* k_cache,
-                          void* v_cache);
+                          const CUtensorMap& tm_x, const CUtensorMap& tm_w, const int32_t* q_pos,
+                          void* k_cache, void* v_cache);
+cudaError_t launch_gemm_tc(int num_sms, cudaStream_t st, const CUtensorMap& tm_a,
+                           const CUtensorMap& tm_b0, const CUtensorMap& tm_b1, GemmParams p);
+size_t gemm_tc_smem_bytes();
+// model_kernels.cu
+cudaError_t launch_rmsnorm(cudaStream_t st, const __nv_bfloat16* x, const int32_t* rows, int n_rows,
+                           int D, const __nv_bfloat16* g, float eps, __nv_bfloat16* y);
+cudaError_t launch_lmhead_reduce(cudaStream_t st, const float* partials, int R, int num_n,
+                                 float threshold, int32_t* token, float* confidence,
+                                 uint8_t* accept);
+// The body of fc_step with the projection weights' tensor map given (the
+// model runs every layer through one handle's workspace).
+fc_status step_impl(fc_handle* h, const CUtensorMap* tm_w, void* stream, int batch, const void* x, const int32_t* q_pos, const int32_t* cu_seqlens_q,
+                    const int32_t* cu_seqlens_k, int total_q, int total_k, void* k_cache,
+                    void* v_cache, void* out, float* importance, int accumulate);
 cudaError_t launch_attn_tc(const fc_handle* h, cudaStream_t st, const StepShape& s,
                            const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                            const int32_t* cu_q, const int32_t* cu_k, void* out,

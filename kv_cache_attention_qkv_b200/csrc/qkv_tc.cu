@@ -320,8 +320,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 size_t qkv_tc_smem_bytes() { return STAGES * STAGE_BYTES + sizeof(Bars) + 1024; }
 
 cudaError_t launch_qkv_tc(const fc_handle* h, cudaStream_t st, const StepShape& s,
-                          const CUtensorMap& tm_x, const int32_t* q_pos, void* k_cache,
-                          void* v_cache) {
+                          const CUtensorMap& tm_x, const CUtensorMap& tm_w, const int32_t* q_pos,
+                          void* k_cache, void* v_cache) {
   QkvParams p;
   p.T = s.T;
   p.S = s.S;
@@ -377,7 +377,7 @@ cudaError_t launch_qkv_tc(const fc_handle* h, cudaStream_t st, const StepShape& 
     cfg.gridDim = dim3(2 * pairs, 1, 1);
   }
   cudaGetLastError();
-  e = cudaLaunchKernelEx(&cfg, qkv_tc_kernel, tm_x, h->tm_w, p);
+  e = cudaLaunchKernelEx(&cfg, qkv_tc_kernel, tm_x, tm_w, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -250,3 +250,125 @@ def describe(name: str) -> Dict[str, object]:
                           cache="200,333", query="40+16, 64+64"),
     }
     return table[name]
+
+
+# --------------------------------------------------------------------------
+# Model-step inputs (the decoder stack around the Flash-Cache layer)
+
+MODEL_WORKLOADS = ("model_small", "model_llada8b")
+
+
+@dataclasses.dataclass
+class ModelInputs:
+    """One model step's inputs, drawn directly on a torch device (bf16).
+
+    ``x_mask`` and ``x_draft`` are the two Flash-Verify views of the query
+    rows: the tracked rows are the same in both; the window rows are one
+    shared [MASK] vector in the first and one vector per row (the drafts) in
+    the second.  ``head_rows`` are the packed indices of the window rows, the
+    rows the LM head scores.
+    """
+
+    name: str
+    hidden: int
+    n_heads: int
+    head_dim: int
+    rope_theta: float
+    intermediate: int
+    vocab: int
+    n_layers: int
+    layers: list  # per layer: dict of bf16 tensors (fc_layer_weights names)
+    final_norm: object
+    lm_head: object
+    x_mask: object
+    x_draft: object
+    k_caches: list
+    v_caches: list
+    q_pos: np.ndarray
+    cu_seqlens_q: np.ndarray
+    cu_seqlens_k: np.ndarray
+    head_rows: np.ndarray
+    cand_lo: np.ndarray
+    cand_hi: np.ndarray
+    topk: np.ndarray
+    window_start: np.ndarray
+    window_len: np.ndarray
+
+    @property
+    def batch(self) -> int:
+        return int(self.cu_seqlens_q.shape[0] - 1)
+
+    @property
+    def total_q(self) -> int:
+        return int(self.cu_seqlens_q[-1])
+
+    @property
+    def total_k(self) -> int:
+        return int(self.cu_seqlens_k[-1])
+
+
+def generate_model(name: str, device="cuda", seed: Optional[int] = None) -> ModelInputs:
+    """Draw a model workload on ``device`` with a seeded torch generator.
+
+    * ``model_small``: 2 layers, hidden 256, 2 heads x 128, SwiGLU 512, vocab
+      1000 (a ragged last vocabulary tile), B=2 with caches of 300 and 200 rows,
+      24/16 tracked + 16 window rows; weights N(0, 0.0625).
+    * ``model_llada8b``: the LLaDA-8B shapes of the pages' model (32 layers,
+      hidden 4096, 32 heads x 128, SwiGLU 12288, vocab 126464), B=32, caches
+      of 1536 rows, 64 tracked + 64 window rows; weights N(0, 0.02).
+    Norm weights are 1 + N(0, 0.1); prior caches N(0, 1); input rows N(0, 1).
+    """
+    import torch
+
+    if name not in MODEL_WORKLOADS:
+        raise ValueError(f"unknown model workload {name!r}; known: {MODEL_WORKLOADS}")
+    if seed is None:
+        seed = 200 + MODEL_WORKLOADS.index(name)
+    rng = np.random.default_rng(seed)
+    if name == "model_small":
+        D, H, d, I, V, NL, theta, w_std = 256, 2, 128, 512, 1000, 2, 5.0e5, 0.0625
+        lens, windows, budgets = [300, 200], [16, 16], [24, 16]
+        starts = [208, 160]
+    else:
+        D, H, d, I, V, NL, theta, w_std = 4096, 32, 128, 12288, 126464, 32, 5.0e5, 0.02
+        B = 32
+        lens, windows, budgets = [1536] * B, [64] * B, [64] * B
+        starts = [int(1024 + 64 * rng.integers(0, (1536 - 1024) // 64)) for _ in range(B)]
+    q_pos, cu_q, cu_k = _layout(rng, lens, windows, budgets, starts)
+    T, S = int(cu_q[-1]), int(cu_k[-1])
+    head_rows = np.concatenate([np.arange(cu_q[b + 1] - w, cu_q[b + 1])
+                                for b, w in enumerate(windows)]).astype(np.int32)
+
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    bf = torch.bfloat16
+
+    def normal(shape, std):
+        return (torch.randn(shape, generator=gen, device=device) * std).to(bf)
+
+    def norm_w():
+        return (1.0 + 0.1 * torch.randn((D,), generator=gen, device=device)).to(bf)
+
+    layers = []
+    for _ in range(NL):
+        layers.append({"attn_norm": norm_w(), "w_qkv": normal((3 * H * d, D), w_std),
+                       "w_o": normal((D, H * d), w_std), "mlp_norm": norm_w(),
+                       "w_gate": normal((I, D), w_std), "w_up": normal((I, D), w_std),
+                       "w_down": normal((D, I), w_std)})
+    final_norm = norm_w()
+    lm_head = normal((V, D), w_std)
+    x_draft = normal((T, D), 1.0)
+    x_mask = x_draft.clone()
+    mask_vec = normal((D,), 1.0)
+    x_mask[torch.from_numpy(head_rows).long().to(device)] = mask_vec
+    k_caches = [normal((S, H, d), 1.0) for _ in range(NL)]
+    v_caches = [normal((S, H, d), 1.0) for _ in range(NL)]
+    starts_a = np.asarray(starts, np.int32)
+    return ModelInputs(
+        name=name, hidden=D, n_heads=H, head_dim=d, rope_theta=float(theta), intermediate=I,
+        vocab=V, n_layers=NL, layers=layers, final_norm=final_norm, lm_head=lm_head,
+        x_mask=x_mask, x_draft=x_draft, k_caches=k_caches, v_caches=v_caches, q_pos=q_pos,
+        cu_seqlens_q=cu_q, cu_seqlens_k=cu_k, head_rows=head_rows,
+        cand_lo=np.zeros(len(lens), np.int32), cand_hi=starts_a.copy(),
+        topk=np.asarray(budgets, np.int32), window_start=starts_a,
+        window_len=np.asarray(windows, np.int32))
