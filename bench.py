@@ -18,6 +18,7 @@ the host cores instead (the deliberately slow baseline arm).
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -421,6 +422,96 @@ def run_reference(args):
     }
 
 
+def run_model(args):
+    """The LLaDA-8B-shaped model step (32 decoder layers around the Flash-Cache
+    layer, LM head over the window rows, Flash-Verify confidence), both views
+    (the [MASK] view, then the draft view) per step, then the reselection of
+    the tracked positions from the draft view's importance summed over layers."""
+    import torch
+
+    from kv_cache_attention_qkv_b200 import FlashCacheModel, workloads
+    from kv_cache_attention_qkv_b200.binding import load_library
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    mi = workloads.generate_model("model_llada8b", device=dev)
+    n = np.diff(mi.cu_seqlens_q)
+    L = np.diff(mi.cu_seqlens_k)
+    R, T, S, B = len(mi.head_rows), mi.total_q, mi.total_k, mi.batch
+    K = int(mi.topk.max())
+    model = FlashCacheModel(mi.layers, mi.final_norm, mi.lm_head, hidden=mi.hidden,
+                            n_heads=mi.n_heads, head_dim=mi.head_dim, rope_theta=mi.rope_theta,
+                            intermediate=mi.intermediate, max_batch=B, max_total_q=T,
+                            max_total_k=S, max_seqlen_q=int(n.max()), max_pos=int(L.max()),
+                            max_topk=K, max_head_rows=R)
+    lib = load_library()
+    i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+    qp, cq, ck, hr = i32(mi.q_pos), i32(mi.cu_seqlens_q), i32(mi.cu_seqlens_k), i32(mi.head_rows)
+    lo, hi, kps = i32(mi.cand_lo), i32(mi.cand_hi), i32(mi.topk)
+    imp = torch.empty((S,), device=dev)
+    outs = {v: (torch.empty((R,), dtype=torch.int32, device=dev), torch.empty((R,), device=dev),
+                torch.empty((R,), dtype=torch.uint8, device=dev)) for v in ("mask", "draft")}
+    tracked = torch.empty((B, K), dtype=torch.int32, device=dev)
+    layer_h = lib.fc_model_layer_handle(model._m)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        model.step(mi.x_mask, qp, cq, ck, mi.k_caches, mi.v_caches, head_rows=hr,
+                   token=outs["mask"][0], confidence=outs["mask"][1], accept=outs["mask"][2])
+        n1 = model.last_launch_count
+        model.step(mi.x_draft, qp, cq, ck, mi.k_caches, mi.v_caches, head_rows=hr, importance=imp,
+                   token=outs["draft"][0], confidence=outs["draft"][1], accept=outs["draft"][2])
+        n2 = model.last_launch_count
+        st = lib.fc_topk_tracked(layer_h, ctypes.c_void_p(stream.cuda_stream), B, S,
+                                 ctypes.c_void_p(imp.data_ptr()), ctypes.c_void_p(ck.data_ptr()),
+                                 ctypes.c_void_p(lo.data_ptr()), ctypes.c_void_p(hi.data_ptr()),
+                                 ctypes.c_void_p(kps.data_ptr()), K,
+                                 ctypes.c_void_p(tracked.data_ptr()))
+        if st != 0:
+            raise RuntimeError(f"fc_topk_tracked: {st}")
+        return n1 + n2 + lib.fc_last_launch_count(layer_h)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if model.get_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches = 0
+    with ClockSampler(0) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            launches += step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if model.get_error() != 0:
+        raise RuntimeError("device error word set during the timed steps")
+    ms = e0.elapsed_time(e1) / args.steps
+    D, H, d, I, V, NL = mi.hidden, mi.n_heads, mi.head_dim, mi.intermediate, mi.vocab, mi.n_layers
+    per_layer = (2.0 * T * D * 3 * H * d + 4.0 * H * d * float((n * L).sum()) + 2.0 * T * H * d * D
+                 + 2.0 * T * D * 2 * I + 2.0 * T * I * D)
+    flops = 2 * (NL * per_layer + 2.0 * R * D * V)  # two views
+    peaks = _peaks()
+    achieved = flops / (ms / 1e3) / 1e12
+    model.close()
+    return {
+        "metric": "query-tokens/s per model step (32 layers, two Flash-Verify views)",
+        "value": T / (ms / 1e3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random-init weights)",
+        "config": {"workload": "model_llada8b", "layers": NL, "hidden": D, "heads": H,
+                   "head_dim": d, "intermediate": I, "vocab": V, "batch": B, "seq_len": int(L.max()),
+                   "query_rows_per_seq": int(n.max()), "head_rows": R, "views": 2,
+                   "l2": "working set (weights 9 GB, caches 26 GB) far above L2"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
+                     "flops_per_step": flops, "traffic": None,
+                     "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json sustained)"},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+
+
 # Sweep axes (the pages' measured axes, throughput side): batch size at the
 # headline query and cache, query size beta_m at batch 32, cache length at
 # batch 32 and beta_m 128.
@@ -440,11 +531,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of oracle time for cpu_baseline (0 = skip)")
+    ap.add_argument("--model", action="store_true",
+                    help="time the 32-layer model step around the layer (one JSON line)")
     ap.add_argument("--sweep", choices=sorted(SWEEPS) + ["all"], default=None,
                     help="time every point of a sweep axis (one JSON line per point, no cpu_baseline)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.model:
+        print(json.dumps(run_model(args)), flush=True)
+        return
     if args.sweep is not None:
         if args.impl != "ours":
             ap.error("--sweep times this implementation only")
