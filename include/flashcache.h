@@ -372,6 +372,51 @@ FC_API fc_status fc_model_step(fc_model* m, void* stream, int batch, const void*
  * kernels). */
 FC_API fc_handle* fc_model_layer_handle(fc_model* m);
 
+/*
+ * fc_decode_iteration — one draft-and-verify decode iteration of every
+ * sequence (Flash-Verify: the model is its own drafter and verifier; draft and
+ * [MASK] tokens are checked through two views; every prediction that meets
+ * the confidence threshold is accepted in the same iteration; the tracked
+ * positions are reselected by importance).  All on the device, on `stream`:
+ *  1. query of sequence b = its K tracked positions, then the W positions of
+ *     its window [window_start[b], window_start[b] + W);
+ *  2. [MASK] view: undecided window rows read embed[mask_id]; draft view: they
+ *     read embed[draft] (embed[mask_id] with no draft); decided rows read
+ *     embed[token] in both; one fc_model_step per view, the LM head on the
+ *     window rows, the draft view's importance summed over layers;
+ *  3. an undecided window position is accepted when the [MASK] view's
+ *     confidence >= threshold (its token), or when the draft view predicts the
+ *     position's draft with confidence >= threshold; if nothing in a window is
+ *     accepted, its undecided position with the highest [MASK]-view confidence
+ *     is (lowest position on ties); undecided positions get the [MASK] view's
+ *     prediction as their next draft; a fully decided window advances by W
+ *     when the next window still ends inside the span (window_start + 2W <=
+ *     gen_end);
+ *  4. tracked := the top-K positions of [0, window_start) by importance.
+ *   cu_seqlens_k, total_k      dev, as for fc_step; k_caches/v_caches as for
+ *                              fc_model_step (the caches keep the draft view's
+ *                              rows: both views write the same rows and the
+ *                              draft view runs second).
+ *   embed          dev, [V, D] bf16 (V = the model's vocab).
+ *   mask_id        0 <= mask_id < V.
+ *   n_tracked (K)  <= max_topk; window (W) >= 1; B * (K + W) <= max_total_q and
+ *                  B * W <= max_head_rows of the model's config.
+ *   tracked        dev, int32 [B, K], in/out: positions, each in [0, ws) (so
+ *                  window_start >= K); entries past the candidates are -1.
+ *   window_start   dev, int32 [B], in/out.   gen_end  dev, int32 [B]: end of
+ *                  the generated span (window_start + W <= gen_end <= L_b).
+ *   tokens, draft  dev, int32 [S] (one entry per cache row, -1 = none), in/out.
+ *   n_accepted     dev, int32 [B], out: tokens accepted this iteration.
+ * Device-side checks (positions, ids) set the layer handle's error word.
+ */
+FC_API fc_status fc_decode_iteration(fc_model* m, void* stream, int batch,
+                                     const int32_t* cu_seqlens_k, int total_k,
+                                     void* const* k_caches, void* const* v_caches,
+                                     const void* embed, int mask_id, int n_tracked, int window,
+                                     int32_t* tracked, int32_t* window_start,
+                                     const int32_t* gen_end, int32_t* tokens, int32_t* draft,
+                                     int32_t* n_accepted);
+
 /* Release the model, its layer handle and workspace (NULL is a no-op). */
 FC_API void fc_model_destroy(fc_model* m);
 

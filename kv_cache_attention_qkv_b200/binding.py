@@ -25,7 +25,8 @@ DEVERR = {0x01: "POS_RANGE", 0x02: "POS_DUP", 0x04: "SEQLENS", 0x08: "CAND", 0x1
 EXPORTED = ("fc_create", "fc_step", "fc_topk_tracked", "fc_step_host", "fc_host_sync",
             "fc_get_error", "fc_last_launch_count", "fc_profile", "fc_profile_read",
             "fc_attention_noalloc", "fc_selftest_wait_timeout", "fc_destroy", "fc_status_str",
-            "fc_model_create", "fc_model_step", "fc_model_layer_handle", "fc_model_destroy")
+            "fc_model_create", "fc_model_step", "fc_model_layer_handle", "fc_model_destroy",
+            "fc_decode_iteration")
 PROFILE_SLOTS = ("prep", "qkv_rope_scatter", "attention", "importance_finalize", "topk")
 
 
@@ -105,6 +106,9 @@ def load_library(path: Optional[str] = None):
     lib.fc_model_layer_handle.restype = vp
     lib.fc_model_destroy.argtypes = [vp]
     lib.fc_model_destroy.restype = None
+    lib.fc_decode_iteration.argtypes = [vp, vp, c_int, vp, c_int, vp, vp, vp, c_int, c_int, c_int,
+                                        vp, vp, vp, vp, vp, vp]
+    lib.fc_decode_iteration.restype = c_int
     lib.fc_status_str.argtypes = [c_int]
     lib.fc_status_str.restype = ctypes.c_char_p
     if path is None:
@@ -347,6 +351,22 @@ class FlashCacheModel:
                                     _ptr(confidence), _ptr(accept), _ptr(h_out))
         if st != 0:
             raise FlashCacheError(st, "fc_model_step")
+
+    def decode_iteration(self, cu_seqlens_k, k_caches, v_caches, embed, mask_id: int, tracked,
+                         window_start, gen_end, tokens, draft, n_accepted, window: int,
+                         stream=None) -> None:
+        """Enqueue fc_decode_iteration; tracked is int32 [B, K], the state arrays are
+        int32 device tensors updated in place."""
+        B, K = tracked.shape
+        kp = (ctypes.c_void_p * self.n_layers)(*[t.data_ptr() for t in k_caches])
+        vp_ = (ctypes.c_void_p * self.n_layers)(*[t.data_ptr() for t in v_caches])
+        st = self.lib.fc_decode_iteration(self._m, _stream_handle(stream), B, _ptr(cu_seqlens_k),
+                                          k_caches[0].shape[0], kp, vp_, _ptr(embed), int(mask_id),
+                                          int(K), int(window), _ptr(tracked), _ptr(window_start),
+                                          _ptr(gen_end), _ptr(tokens), _ptr(draft),
+                                          _ptr(n_accepted))
+        if st != 0:
+            raise FlashCacheError(st, "fc_decode_iteration")
 
     def get_error(self) -> int:
         """Wait for the last stream used and return (and clear) the device error word."""

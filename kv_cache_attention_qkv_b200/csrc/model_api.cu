@@ -28,7 +28,20 @@ struct fc_model {
   float* partials = nullptr;
   int num_vn = 0;  // 256-column vocabulary tiles
   CUtensorMap tm_a, tm_oa, tm_s, tm_hr;
+  void* decode_ws[16] = {};  // fc_decode_iteration's workspace (allocated on first use)
 };
+
+namespace fc {
+int model_hidden(const fc_model* m) { return m->cfg.layer.hidden; }
+int model_vocab(const fc_model* m) { return m->cfg.vocab; }
+int model_max_total_q(const fc_model* m) { return m->cfg.layer.max_total_q; }
+int model_max_batch(const fc_model* m) { return m->cfg.layer.max_batch; }
+int model_max_head_rows(const fc_model* m) { return m->cfg.max_head_rows; }
+int model_max_topk(const fc_model* m) { return m->cfg.layer.max_topk; }
+float model_threshold(const fc_model* m) { return m->cfg.threshold; }
+fc_handle* model_layer(fc_model* m) { return m->layer; }
+void** model_decode_ws(fc_model* m) { return m->decode_ws; }
+}  // namespace fc
 
 namespace {
 
@@ -37,6 +50,8 @@ bool al16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
 void free_model(fc_model* m) {
   void* bufs[] = {m->h, m->a, m->o, m->s, m->hr, m->partials};
   for (void* b : bufs)
+    if (b) cudaFree(b);
+  for (void* b : m->decode_ws)
     if (b) cudaFree(b);
   if (m->layer) fc_destroy(m->layer);
   delete m;

@@ -282,6 +282,7 @@ class ModelInputs:
     lm_head: object
     x_mask: object
     x_draft: object
+    embed: object  # [V, D] token embeddings (for decoding); the [MASK] token is V - 1
     k_caches: list
     v_caches: list
     q_pos: np.ndarray
@@ -361,13 +362,15 @@ def generate_model(name: str, device="cuda", seed: Optional[int] = None) -> Mode
     x_mask = x_draft.clone()
     mask_vec = normal((D,), 1.0)
     x_mask[torch.from_numpy(head_rows).long().to(device)] = mask_vec
+    embed = normal((V, D), 1.0)
     k_caches = [normal((S, H, d), 1.0) for _ in range(NL)]
     v_caches = [normal((S, H, d), 1.0) for _ in range(NL)]
     starts_a = np.asarray(starts, np.int32)
     return ModelInputs(
         name=name, hidden=D, n_heads=H, head_dim=d, rope_theta=float(theta), intermediate=I,
         vocab=V, n_layers=NL, layers=layers, final_norm=final_norm, lm_head=lm_head,
-        x_mask=x_mask, x_draft=x_draft, k_caches=k_caches, v_caches=v_caches, q_pos=q_pos,
+        x_mask=x_mask, x_draft=x_draft, embed=embed, k_caches=k_caches, v_caches=v_caches,
+        q_pos=q_pos,
         cu_seqlens_q=cu_q, cu_seqlens_k=cu_k, head_rows=head_rows,
         cand_lo=np.zeros(len(lens), np.int32), cand_hi=starts_a.copy(),
         topk=np.asarray(budgets, np.int32), window_start=starts_a,

@@ -25,8 +25,8 @@ Readings taken where the pages are silent:
   (lowest position on ties), so every iteration decodes at least one token;
 * the drafts of the positions still undecided become the [MASK] view's
   predictions;
-* when the whole window is decided it advances by W (while it stays inside
-  the generated span) and the new window has no drafts;
+* when the whole window is decided it advances by W if the next window lies
+  inside the generated span, and the new window has no drafts;
 * the tracked positions are then reselected: the top-K positions of
   [0, ws) by the draft view's importance (summed over layers).
 """
@@ -75,7 +75,7 @@ def accept_and_advance(tokens: np.ndarray, draft: np.ndarray, ws: int, W: int, g
     still = tokens[win] < 0
     draft[win[still]] = tok_m[still]
     draft[win[~still]] = -1
-    if not still.any() and ws + W < gen_end:
+    if not still.any() and ws + 2 * W <= gen_end:  # the next window fits in the span
         ws = ws + W
         draft[ws:ws + W] = -1
     return {"tokens": tokens, "draft": draft, "ws": ws, "n_accepted": n_acc}

@@ -53,3 +53,14 @@ def test_decided_positions_are_left_alone():
              td=[9, 9], cd=[0.99, 0.99])
     # pos 2 is decided already (token 3) whatever the views say; pos 3's draft 9 is verified
     assert list(r["tokens"]) == [1, 2, 3, 9] and r["n_accepted"] == 1
+
+
+def test_window_does_not_advance_past_the_span():
+    # span [2, 7): after the window [2, 4) the next one [4, 6) fits, after [4, 6) the
+    # next one [6, 8) would not
+    r = _acc([1, 2, -1, -1, -1, -1, -1], [-1] * 7, 2, 2, 7, tm=[3, 4], cm=[0.95, 0.97],
+             td=[0, 0], cd=[0.0, 0.0])
+    assert r["ws"] == 4
+    r = _acc([1, 2, 3, 4, -1, -1, -1], [-1] * 7, 4, 2, 7, tm=[5, 6], cm=[0.95, 0.97],
+             td=[0, 0], cd=[0.0, 0.0])
+    assert r["ws"] == 4
