@@ -512,6 +512,75 @@ def run_model(args):
     }
 
 
+def run_decode(args):
+    """Draft-and-verify decode iterations of the LLaDA-8B-shaped model: per
+    iteration both views of the 32-layer model step, acceptance, window
+    advance and reselection, all on the device.  Random weights never reach
+    the 0.9 threshold, so each iteration decodes one token per sequence."""
+    import torch
+
+    from kv_cache_attention_qkv_b200 import FlashCacheModel, workloads
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    mi = workloads.generate_model("model_llada8b", device=dev)
+    B, K, W = mi.batch, 64, 64
+    L = np.diff(mi.cu_seqlens_k)
+    model = FlashCacheModel(mi.layers, mi.final_norm, mi.lm_head, hidden=mi.hidden,
+                            n_heads=mi.n_heads, head_dim=mi.head_dim, rope_theta=mi.rope_theta,
+                            intermediate=mi.intermediate, max_batch=B, max_total_q=B * (K + W),
+                            max_total_k=mi.total_k, max_seqlen_q=K + W, max_pos=int(L.max()),
+                            max_topk=K, max_head_rows=B * W)
+    rng = np.random.default_rng(11)
+    prompt = np.full(B, 1024, np.int64)  # 1024 prompt rows, 512 generated
+    tokens = np.full(mi.total_k, -1, np.int32)
+    tracked = np.zeros((B, K), np.int32)
+    for b in range(B):
+        k0 = mi.cu_seqlens_k[b]
+        tokens[k0:k0 + prompt[b]] = rng.integers(0, mi.vocab - 1, size=prompt[b])
+        tracked[b] = np.sort(rng.choice(prompt[b], size=K, replace=False))
+    i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+    st = [i32(tokens), i32(np.full(mi.total_k, -1)), i32(tracked), i32(prompt), i32(np.zeros(B))]
+    gen_end, cu_k = i32(L), i32(mi.cu_seqlens_k)
+    stream = torch.cuda.current_stream()
+
+    def iteration():
+        model.decode_iteration(cu_k, mi.k_caches, mi.v_caches, mi.embed, mi.vocab - 1, st[2],
+                               st[3], gen_end, st[0], st[1], st[4], W)
+        return model.last_launch_count
+
+    for _ in range(args.warmup):
+        iteration()
+    torch.cuda.synchronize()
+    if model.get_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    decided0 = int((st[0] >= 0).sum().item())
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches = 0
+    with ClockSampler(0) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            launches += iteration()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if model.get_error() != 0:
+        raise RuntimeError("device error word set during the timed iterations")
+    decoded = int((st[0] >= 0).sum().item()) - decided0
+    ms = e0.elapsed_time(e1) / args.steps
+    model.close()
+    return {
+        "metric": "decoded tokens/s (draft-and-verify iterations, 32-layer model, both views)",
+        "value": decoded / (ms * args.steps / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (random-init weights: one token per sequence per iteration)",
+        "config": {"workload": "model_llada8b", "batch": B, "tracked": K, "window": W,
+                   "prompt": 1024, "seq_len": int(L.max()), "threshold": 0.9,
+                   "decoded_tokens": decoded, "iterations": args.steps},
+        "gpu_launches": launches, "clocks": clk.summary(),
+    }
+
+
 # Sweep axes (the pages' measured axes, throughput side): batch size at the
 # headline query and cache, query size beta_m at batch 32, cache length at
 # batch 32 and beta_m 128.
@@ -531,6 +600,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of oracle time for cpu_baseline (0 = skip)")
+    ap.add_argument("--decode", action="store_true",
+                    help="time draft-and-verify decode iterations of the model (one JSON line)")
     ap.add_argument("--model", action="store_true",
                     help="time the 32-layer model step around the layer (one JSON line)")
     ap.add_argument("--sweep", choices=sorted(SWEEPS) + ["all"], default=None,
@@ -540,6 +611,9 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.model:
         print(json.dumps(run_model(args)), flush=True)
+        return
+    if args.decode:
+        print(json.dumps(run_decode(args)), flush=True)
         return
     if args.sweep is not None:
         if args.impl != "ours":
