@@ -6,7 +6,8 @@
 // paragraph: only newly decoded tokens and a few key positions chosen by
 // attention importance are refreshed).
 //
-// topk_tracked: one CTA per sequence.  An exact radix select (four 8-bit
+// topk_tracked: one CTA per sequence; up to 8192 candidates are staged in
+// shared memory as keys.  An exact radix select (four 8-bit
 // digits of an order-preserving 32-bit key) finds the k-th largest score; all
 // larger scores are kept, equal ones in position order until k are kept, and
 // the kept set is sorted by (score desc, position asc).  The result does not
@@ -37,6 +38,7 @@ __device__ __forceinline__ uint32_t fkey(float f) {
 
 constexpr int TK_THREADS = 512;
 constexpr int TK_MAXK = 1024;
+constexpr int TK_STAGE = 8192;  // candidate keys staged in shared memory (32 KiB)
 
 __global__ void __launch_bounds__(TK_THREADS) topk_kernel(
     int B, const float* __restrict__ imp, const int32_t* __restrict__ cu_k,
@@ -47,6 +49,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(
   __shared__ unsigned long long sel[TK_MAXK];
   __shared__ int sh_digit, sh_remaining, sh_nsel, sh_run;
   __shared__ int warp_cnt[TK_THREADS / 32];
+  __shared__ uint32_t skey[TK_STAGE];
 
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t* row = tracked + (size_t)b * k;
@@ -66,6 +69,13 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(
   const int n = hi - lo;
   const int want = min(kb, n);
   const float* sc = imp + k0 + lo;
+  // up to TK_STAGE candidates are read from global memory once, as keys
+  const bool staged = n <= TK_STAGE;
+  if (staged && want > 0) {
+    for (int i = tid; i < n; i += TK_THREADS) skey[i] = fkey(sc[i]);
+    __syncthreads();
+  }
+  auto key_of = [&](int i) { return staged ? skey[i] : fkey(sc[i]); };
 
   // ---- radix select of the want-th largest key
   uint32_t prefix = 0u, mask = 0u;
@@ -75,7 +85,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(
       for (int i = tid; i < 256; i += TK_THREADS) hist[i] = 0u;
       __syncthreads();
       for (int i = tid; i < n; i += TK_THREADS) {
-        const uint32_t key = fkey(sc[i]);
+        const uint32_t key = key_of(i);
         if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1u);
       }
       __syncthreads();
@@ -126,7 +136,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(
       uint32_t key = 0u;
       bool gt = false, eq = false;
       if (i < n) {
-        key = fkey(sc[i]);
+        key = key_of(i);
         gt = key > thr;
         eq = key == thr;
       }
