@@ -101,3 +101,69 @@ def test_valid_config_without_a_device_reports_cuda_error(lib):
 def test_binding_refuses_to_run_without_the_library(tmp_path):
     with pytest.raises(binding.FlashCacheError):
         binding.load_library(str(tmp_path / "missing.so"))
+
+
+def _mcfg(**over):
+    layer = _cfg(hidden=256, n_heads=2, head_dim=128, dtype=binding.FC_DTYPE_BF16)
+    base = dict(layer=layer, n_layers=2, intermediate=512, vocab=1000, max_head_rows=8,
+                rms_eps=1e-5, threshold=0.9)
+    base.update(over)
+    return binding.FcModelConfig(**base)
+
+
+def _weights(n, addr=0x1000):
+    arr = (binding.FcLayerWeights * n)()
+    for i in range(n):
+        for name in binding.LAYER_WEIGHT_NAMES:
+            setattr(arr[i], name, addr)
+    return arr
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(n_layers=0), -1), (dict(intermediate=0), -1), (dict(vocab=0), -1),
+    (dict(max_head_rows=0), -1), (dict(rms_eps=-1.0), -1), (dict(threshold=float("nan")), -1),
+    (dict(intermediate=500), -2),  # SwiGLU tiles are 128 features wide
+])
+def test_model_create_rejects_bad_config_before_touching_the_device(lib, over, expect):
+    m = ctypes.c_void_p()
+    cfg = _mcfg(**over)
+    st = lib.fc_model_create(ctypes.byref(cfg), _weights(max(cfg.n_layers, 1)),
+                             ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1000), ctypes.byref(m))
+    assert st == expect and not m.value
+
+
+def test_model_create_rejects_unsupported_layer_shapes(lib):
+    m = ctypes.c_void_p()
+    for layer in (_cfg(hidden=256, n_heads=2, head_dim=128),  # fp32
+                  _cfg(hidden=256, n_heads=3, head_dim=128, dtype=binding.FC_DTYPE_BF16),
+                  _cfg(hidden=320, n_heads=2, head_dim=128, dtype=binding.FC_DTYPE_BF16),
+                  _cfg(hidden=256, n_heads=4, head_dim=64, dtype=binding.FC_DTYPE_BF16)):
+        cfg = _mcfg(layer=layer)
+        st = lib.fc_model_create(ctypes.byref(cfg), _weights(2), ctypes.c_void_p(0x1000),
+                                 ctypes.c_void_p(0x1000), ctypes.byref(m))
+        assert st == -2 and not m.value
+
+
+def test_model_create_rejects_null_and_misaligned_weights(lib):
+    m = ctypes.c_void_p()
+    cfg = _mcfg()
+    assert lib.fc_model_create(ctypes.byref(cfg), None, ctypes.c_void_p(0x1000),
+                               ctypes.c_void_p(0x1000), ctypes.byref(m)) == -1
+    assert lib.fc_model_create(ctypes.byref(cfg), _weights(2, 0x1008), ctypes.c_void_p(0x1000),
+                               ctypes.c_void_p(0x1000), ctypes.byref(m)) == -1
+    assert lib.fc_model_create(ctypes.byref(cfg), _weights(2), None, ctypes.c_void_p(0x1000),
+                               ctypes.byref(m)) == -1
+
+
+def test_model_and_host_step_calls_on_null_handles_are_rejected(lib):
+    vp = ctypes.c_void_p
+    arr = (ctypes.c_void_p * 2)(16, 16)
+    assert lib.fc_model_step(None, None, 1, vp(16), vp(16), vp(16), vp(16), 1, 1, arr, arr, None,
+                             0, None, None, None, None, None) == -1
+    assert lib.fc_decode_iteration(None, None, 1, vp(16), 1, arr, arr, vp(16), 0, 1, 1, vp(16),
+                                   vp(16), vp(16), vp(16), vp(16), vp(16)) == -1
+    assert lib.fc_step_host(None, None, 1, vp(16), vp(16), vp(16), vp(16), 1, 1, vp(16), vp(16),
+                            vp(16), vp(16), None, 1, vp(16), vp(16)) == -1
+    assert lib.fc_host_sync(None, None) == -1
+    assert lib.fc_model_layer_handle(None) is None
+    lib.fc_model_destroy(None)  # no-op
