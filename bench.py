@@ -322,10 +322,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": inp.dtype, "data": "synthetic",
-            "config": {"workload": args.workload, "batch": B, "seq_len": int(np.diff(inp.cu_seqlens_k).max()),
-                       "query_rows_per_seq": int(np.diff(inp.cu_seqlens_q).max()), "hidden": inp.hidden,
-                       "heads": H, "head_dim": d, "topk": K, "total_q": T, "total_k": S,
-                       "l2": "flushed between steps (256 MiB write)", "parallelism": f"sequence-sharded x{ws}"},
+            "config": _step_config(args.workload, inp, ws),
             "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                          "frac": achieved / peak, "traffic": traffic.get(dom),
                          "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst)"},
@@ -356,6 +353,15 @@ def _oracle_threads():
         return int(max(n)) if n else os.cpu_count()
     except Exception:
         return os.cpu_count()
+
+
+def _step_config(workload, inp, ws):
+    """The workload description both arms print (the same keys at every N)."""
+    return {"workload": workload, "batch": inp.batch, "seq_len": int(np.diff(inp.cu_seqlens_k).max()),
+            "query_rows_per_seq": int(np.diff(inp.cu_seqlens_q).max()), "hidden": inp.hidden,
+            "heads": inp.n_heads, "head_dim": inp.head_dim, "topk": int(inp.topk.max()),
+            "total_q": inp.total_q, "total_k": inp.total_k,
+            "l2": "flushed between steps (256 MiB write)", "parallelism": f"sequence-sharded x{ws}"}
 
 
 def cpu_baseline(inp, budget_s: float = 12.0):
@@ -415,9 +421,10 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": args.workload, "sample_per_step": "one sequence (its query rows)"},
+        "config": _step_config(args.workload, inp, ws),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
-                         "sample": f"{args.steps} sequence(s) of workload {args.workload}, one per step"},
+                         "sample": f"{args.steps} sequence(s) of workload {args.workload}, one per step "
+                                   "(each step times one sequence's query rows)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
