@@ -170,3 +170,21 @@ def test_acceptance_threshold_branch():
     r = mo.model_step_sequence(x, [], fn, np.zeros((V, D)), np.array([0, 1]), [], [],
                                np.array([0, 1]), 2, 16, 1e4, act_dtype=None, cache_dtype=None)
     assert not r["accept"].any()
+
+
+def test_lm_head_reads_the_final_normed_stream():
+    """With no layers the LM head sees rms_norm(x) * g_final: the planted
+    logit is z * rms_norm(x)[0], close to z * sqrt(D) at any scale of x, and
+    the confidence has the corresponding closed form."""
+    D, V, z = 32, 40, 0.5
+    wlm = np.zeros((V, D))
+    wlm[5, 0] = z
+    for s in (0.5, 3.0):
+        x = np.zeros((1, D))
+        x[0, 0] = s  # rms_norm(x)[0] = s / sqrt(s^2 / D + eps), about sqrt(D)
+        t = z * s / math.sqrt(s * s / D + 1e-5)
+        want = math.exp(t) / (math.exp(t) + V - 1)
+        r = mo.model_step_sequence(x, [], np.ones(D), wlm, np.array([0]), [], [], np.array([0]),
+                                   2, 16, 1e4, act_dtype=None, cache_dtype=None)
+        assert r["token"][0] == 5
+        np.testing.assert_allclose(r["confidence"][0], want, rtol=1e-12)
