@@ -392,7 +392,8 @@ FC_API fc_handle* fc_model_layer_handle(fc_model* m);
  *     prediction as their next draft; a fully decided window advances by W
  *     when the next window still ends inside the span (window_start + 2W <=
  *     gen_end);
- *  4. tracked := the top-K positions of [0, window_start) by importance.
+ *  4. tracked := the top-K positions of [0, window_start) by the draft view's
+ *     importance, window_start as advanced in step 3.
  *   cu_seqlens_k, total_k      dev, as for fc_step; k_caches/v_caches as for
  *                              fc_model_step (the caches keep the draft view's
  *                              rows: both views write the same rows and the
