@@ -44,11 +44,13 @@ _KERNEL_SOURCES = {
 
 
 def _kernel_roofline(name, bound, work, timing, peaks, traffic):
-    """Achieved rate of one kernel (algorithmic work / mean launch time)."""
+    """Achieved rate of one kernel (algorithmic work / mean launch time).  The
+    kernels are timed in the steady state of a sustained load, so a contraction
+    is set against the sustained bf16 GEMM rate."""
     ms, n = timing
     avg_s = ms / max(n, 1) / 1e3
     if bound == "tensor":
-        achieved, peak, unit = work / avg_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        achieved, peak, unit = work / avg_s / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
     else:
         achieved, peak, unit = work / avg_s / 1e9, peaks["hbm_gbs"], "GB/s"
     return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
@@ -104,9 +106,11 @@ def _work(inp):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms; the summary
+    keeps the samples taken between window_start() and window_end() (the load
+    window around the timed steps)."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -114,6 +118,7 @@ class ClockSampler:
         self.idx = gpu_index
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         import tempfile
@@ -129,6 +134,12 @@ class ClockSampler:
         time.sleep(0.3)
         return self
 
+    def window_start(self):
+        self.t0 = time.time()
+
+    def window_end(self):
+        self.t1 = time.time()
+
     def __exit__(self, *exc):
         if self.proc is not None:
             time.sleep(0.2)
@@ -139,16 +150,26 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        import datetime
+
         if self.proc is None or not self.path or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         rows = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
+            if len(parts) >= 10:
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    ts = None
+                rows.append((ts, parts[1:]))
         os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        inside = rows
+        if self.t0 is not None and self.t1 is not None:
+            inside = [r for r in rows if r[0] is not None and self.t0 <= r[0] <= self.t1]
+        window = [r for _, r in (inside or rows)]
 
         def num(v):
             try:
@@ -156,13 +177,18 @@ class ClockSampler:
             except ValueError:
                 return None
 
-        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
-        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
-        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        sm = [num(r[1]) for r in window if num(r[1]) is not None]
+        mx = [num(r[2]) for r in window if num(r[2]) is not None]
+        pw = [num(r[3]) for r in window if num(r[3]) is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "power_w_max": max(pw) if pw else None, "samples": len(rows), "reasons": reasons}
+        reasons = sorted({names[i] for r in window for i in range(4) if r[5 + i].lower() == "active"})
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+               "power_w_max": max(pw) if pw else None, "samples": len(window), "reasons": reasons}
+        if self.t0 is not None and self.t1 is not None:
+            out["window_s"] = round(self.t1 - self.t0, 3)
+            if not inside:
+                out["note"] = "no sample inside the load window; all samples summarised"
+        return out
 
 
 def _dist_env():
@@ -224,41 +250,65 @@ def run_ours(args):
     if layer.get_error() != 0:
         raise RuntimeError("device error word set during warm-up")
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    launches = 0
+    def timed_steps(n):
+        """n steps with an event pair around each, an L2 flush before each."""
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        nl = 0
+        for k in range(n):
+            flush.fill_(float(k))
+            evs[k][0].record(stream)
+            nl += step()
+            evs[k][1].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs], nl
+
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    # burst (context only): the same K steps right after the warm-up, before the
+    # power controller has reacted to the load
+    burst_ms = float(sum(timed_steps(args.steps)[0]))
     with ClockSampler(torch.cuda.current_device()) as clk:
+        # The K timed steps last milliseconds, less than the sampler's period, so
+        # they are taken in the steady state of the load: after about a second
+        # of the same untimed steps.  The sampler's window covers that second,
+        # the timed steps and the per-kernel pass.
+        clk.window_start()
+        soak_t0, soak = time.perf_counter(), 0
+        while time.perf_counter() - soak_t0 < 1.0:
+            flush.fill_(float(soak))
+            step()
+            soak += 1
+            if soak % 32 == 0:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        step_ms, launches = timed_steps(args.steps)
+        if ws > 1:
+            dist.barrier()
+        # Per-kernel durations: the same K steps again with a CUDA event pair
+        # around every kernel on its launching stream (events between kernels
+        # stop the programmatic overlap of neighbouring kernels, so this pass is
+        # not the step-time pass above).
+        layer.profile(True)
+        layer.profile_read()
+        torch.cuda.synchronize()
         for k in range(args.steps):
             flush.fill_(float(k))
-            ev[k][0].record(stream)
-            launches += step()
-            ev[k][1].record(stream)
+            step()
         torch.cuda.synchronize()
-    if ws > 1:
-        dist.barrier()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    # Per-kernel durations: the same K steps again with a CUDA event pair around
-    # every kernel on its launching stream (events between kernels stop the
-    # programmatic overlap of neighbouring kernels, so this pass is not the
-    # step-time pass above).
-    layer.profile(True)
-    layer.profile_read()
-    torch.cuda.synchronize()
-    for k in range(args.steps):
-        flush.fill_(float(k))
-        step()
-    torch.cuda.synchronize()
-    per_kernel = layer.profile_read()
-    layer.profile(False)
+        per_kernel = layer.profile_read()
+        layer.profile(False)
+        clk.window_end()
     total_ms = float(sum(step_ms))
     err = layer.get_error()
     if ws > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        t = torch.tensor([total_ms, burst_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms, burst_ms = float(t[0].item()), float(t[1].item())
 
     # ---- end to end through the public API with host buffers
     x_h = torch.from_numpy(np.ascontiguousarray(inp.x)).to(dt).pin_memory()
@@ -310,13 +360,14 @@ def run_ours(args):
         bound, work = names[dom]
         if bound == "tensor":
             achieved = work / avg_s / 1e12
-            peak = peaks["bf16_tflops"]
+            peak = peaks["bf16_tflops_sustained"]
             unit = "TFLOP/s"
         else:
             achieved = work / avg_s / 1e9
             peak = peaks["hbm_gbs"]
             unit = "GB/s"
-        t_roof = max(wk["flops"] / (peaks["bf16_tflops"] * 1e12), wk["bytes"] / (peaks["hbm_gbs"] * 1e9))
+        t_roof = max(wk["flops"] / (peaks["bf16_tflops_sustained"] * 1e12),
+                     wk["bytes"] / (peaks["hbm_gbs"] * 1e9))
         traffic = _dram_traffic(args.workload)
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
@@ -325,7 +376,8 @@ def run_ours(args):
             "config": _step_config(args.workload, inp, ws),
             "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                          "frac": achieved / peak, "traffic": traffic.get(dom),
-                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst)"},
+                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json: sustained bf16 for "
+                                        "tensor-bound kernels, copy bandwidth for HBM-bound ones)"},
             "kernel_rooflines": {k: _kernel_roofline(k, b, w, per_kernel[k], peaks, traffic.get(k))
                                  for k, (b, w) in names.items()},
             "step_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": ms_per_step * 1e3,
@@ -333,6 +385,9 @@ def run_ours(args):
             "kernels_ms_per_step": {k: v[0] / max(v[1], 1) for k, v in per_kernel.items()},
             "gpu_launches": launches,
             "device_error_word": err,
+            "burst": {"value": tokens / (burst_ms / 1e3), "ms_per_step": burst_ms / args.steps,
+                      "note": "the same K steps right after the warm-up, before the power "
+                              "controller reacts; value and rooflines above are the steady state"},
             "e2e": {"value": T * ws * args.steps / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
             "clocks": clk.summary(),
@@ -486,11 +541,13 @@ def run_model(args):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches = 0
     with ClockSampler(0) as clk:
+        clk.window_start()
         e0.record(stream)
         for _ in range(args.steps):
             launches += step()
         e1.record(stream)
         torch.cuda.synchronize()
+        clk.window_end()
     if model.get_error() != 0:
         raise RuntimeError("device error word set during the timed steps")
     ms = e0.elapsed_time(e1) / args.steps
@@ -565,11 +622,13 @@ def run_decode(args):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches = 0
     with ClockSampler(0) as clk:
+        clk.window_start()
         e0.record(stream)
         for _ in range(args.steps):
             launches += iteration()
         e1.record(stream)
         torch.cuda.synchronize()
+        clk.window_end()
     if model.get_error() != 0:
         raise RuntimeError("device error word set during the timed iterations")
     decoded = int((st[0] >= 0).sum().item()) - decided0
