@@ -202,7 +202,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    from kv_cache_attention_qkv_b200 import FlashCache, workloads
+    from kv_cache_attention_qkv_b200 import FlashCache, shard, workloads
 
     ws, rank, local = _dist_env()
     if ws > 1:
@@ -305,10 +305,8 @@ def run_ours(args):
         clk.window_end()
     total_ms = float(sum(step_ms))
     err = layer.get_error()
-    if ws > 1:
-        t = torch.tensor([total_ms, burst_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, burst_ms = float(t[0].item()), float(t[1].item())
+    if ws > 1:  # the slowest rank sets the time
+        total_ms, burst_ms = shard.max_over_ranks([total_ms, burst_ms], device=dev)
 
     # ---- end to end through the public API with host buffers
     x_h = torch.from_numpy(np.ascontiguousarray(inp.x)).to(dt).pin_memory()
@@ -341,9 +339,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     if ws > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+        e2e_ms = shard.max_over_ranks(e2e_ms, device=dev)
 
     result = None
     if rank == 0:

@@ -36,11 +36,15 @@ def shard_batch(inp, rank: int, world: int):
     )
 
 
-def max_over_ranks(value: float, device=None) -> float:
-    """All-reduce MAX of a scalar over the default process group."""
+def max_over_ranks(value, device=None):
+    """All-reduce MAX over the default process group of a scalar (returns a
+    float) or of a sequence of scalars (returns a list, element-wise)."""
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    many = isinstance(value, (list, tuple))
+    vals = [float(v) for v in value] if many else [float(value)]
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    out = [float(v) for v in t.tolist()]
+    return out if many else out[0]

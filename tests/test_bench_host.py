@@ -1,0 +1,94 @@
+"""Host logic of bench.py that needs no GPU: the clock record's load window,
+the workload description shared by both arms, and the reference arm's JSON
+line under torchrun (rank 0 prints it, the other ranks exit quietly)."""
+import datetime
+import json
+import os
+import socket
+import subprocess
+import sys
+import time
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _write_samples(path, t_first, rows):
+    with open(path, "w") as f:
+        for i, (mhz, watts, cap) in enumerate(rows):
+            ts = datetime.datetime.fromtimestamp(t_first + 0.1 * i).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+            state = "Active" if cap else "Not Active"
+            f.write(f"{ts}, 0, {mhz}, 1965, {watts}, 0x0, Not Active, Not Active, Not Active, {state}\n")
+
+
+def _sampler(tmp_path, rows, window=None):
+    c = bench.ClockSampler(0)
+    c.proc = object()  # stands for a running nvidia-smi
+    c.path = str(tmp_path / "clocks.csv")
+    t_first = time.time()
+    _write_samples(c.path, t_first, rows)
+    if window is not None:
+        c.t0, c.t1 = t_first + window[0], t_first + window[1]
+    return c
+
+
+def test_clock_summary_keeps_only_the_load_window(tmp_path):
+    # idle at 1965 MHz, then 10 samples of load at 1600 MHz under the power cap, then idle
+    rows = [(1965, 120.0, False)] * 5 + [(1600, 960.0, True)] * 10 + [(1965, 150.0, False)] * 5
+    s = _sampler(tmp_path, rows, window=(0.45, 1.45)).summary()
+    assert s["samples"] == 10 and s["sm_mhz"] == 1600.0 and s["reasons"] == ["sw_power_cap"]
+    assert s["sm_max_mhz"] == 1965.0 and s["power_w_max"] == 960.0 and s["window_s"] == 1.0
+
+
+def test_clock_summary_without_a_window_or_samples(tmp_path):
+    rows = [(1965, 120.0, False)] * 3
+    s = _sampler(tmp_path, rows).summary()
+    assert s["samples"] == 3 and s["sm_mhz"] == 1965.0 and s["reasons"] == []
+    # a window that no sample falls in: everything is summarised, and said so
+    s = _sampler(tmp_path, rows, window=(100.0, 101.0)).summary()
+    assert s["samples"] == 3 and "note" in s
+    c = bench.ClockSampler(0)
+    assert c.summary()["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_both_arms_describe_the_workload_alike():
+    from kv_cache_attention_qkv_b200 import workloads
+
+    inp = workloads.generate("tiny_fp32")
+    cfg = bench._step_config("tiny_fp32", inp, 2)
+    assert cfg["workload"] == "tiny_fp32" and cfg["parallelism"] == "sequence-sharded x2"
+    assert (cfg["batch"], cfg["total_q"], cfg["total_k"]) == (inp.batch, inp.total_q, inp.total_k)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+@pytest.mark.timeout(300)
+def test_reference_arm_under_torchrun_prints_one_line():
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py",
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3",
+           "--workload", "tiny_fp32"]
+    p = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=280)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [json.loads(l) for l in p.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = lines[0]
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["steps"] == 1
+    assert line["config"] == bench._step_config("tiny_fp32", _tiny(), 2)
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+def _tiny():
+    from kv_cache_attention_qkv_b200 import workloads
+
+    return workloads.generate("tiny_fp32")

@@ -42,8 +42,9 @@ def _worker(rank, world, port, out_q):
         gathered = [None] * world
         dist.all_gather_object(gathered, (res["out"], res["importance"], tracked))
         slowest = shard.max_over_ranks(10.0 + rank)
+        pair = shard.max_over_ranks([5.0 - rank, 7.0 + 2 * rank])
         if rank == 0:
-            out_q.put((gathered, slowest))
+            out_q.put((gathered, (slowest, pair)))
     finally:
         dist.destroy_process_group()
 
@@ -56,7 +57,7 @@ def test_sharded_oracle_matches_unsharded():
     procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
-    gathered, slowest = q.get(timeout=300)
+    gathered, (slowest, pair) = q.get(timeout=300)
     for p in procs:
         p.join(timeout=120)
         assert p.exitcode == 0
@@ -72,6 +73,7 @@ def test_sharded_oracle_matches_unsharded():
     np.testing.assert_array_equal(np.concatenate([g[1] for g in gathered]), full["importance"])
     np.testing.assert_array_equal(np.concatenate([g[2] for g in gathered]), tracked)
     assert slowest == 11.0
+    assert pair == [5.0, 9.0]  # element-wise over the ranks
 
 
 @pytest.mark.parametrize("batch,world", [(32, 8), (3, 2), (5, 4), (1, 1)])
