@@ -388,7 +388,9 @@ def run_ours(args):
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
             "clocks": clk.summary(),
         }
-        result["cpu_baseline"] = cpu_baseline(inp, budget_s=args.cpu_budget) if args.cpu_budget > 0 else None
+        # the oracle's timing is a single-GPU line's context: rank 0 at N = 1 only
+        result["cpu_baseline"] = (cpu_baseline(inp, budget_s=args.cpu_budget)
+                                  if args.cpu_budget > 0 and ws == 1 else None)
     layer.close()
     if ws > 1:
         dist.barrier()
