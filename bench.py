@@ -198,6 +198,52 @@ def _dist_env():
     return ws, rank, local
 
 
+def _step_result(args, inp, ws, *, total_ms, burst_ms, per_kernel, launches, err, e2e_ms, h2d,
+                 d2h, clocks):
+    """The JSON line of a step run from its measurements (no GPU needed).
+
+    per_kernel: {name: (total ms, launches)} of the per-kernel pass; total_ms,
+    burst_ms, e2e_ms: max over ranks of the K steps' device time."""
+    peaks = _peaks()
+    wk = _work(inp)
+    T = inp.total_q
+    ms_per_step = total_ms / args.steps
+    tokens = T * ws * args.steps
+    value = tokens / (total_ms / 1e3)
+    # dominant kernel by measured share
+    names = {"qkv_rope_scatter": ("tensor", wk["qkv_flops"]), "attention": ("hbm", wk["attn_bytes"])}
+    dom = max(names, key=lambda k: per_kernel[k][0])
+    traffic = _dram_traffic(args.workload)
+    rl = _kernel_roofline(dom, *names[dom], per_kernel[dom], peaks, traffic.get(dom))
+    t_roof = max(wk["flops"] / (peaks["bf16_tflops_sustained"] * 1e12),
+                 wk["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": inp.dtype, "data": "synthetic",
+        "config": _step_config(args.workload, inp, ws),
+        "roofline": {"kernel": dom, "bound": rl["bound"], "achieved": rl["achieved"],
+                     "peak": rl["peak"], "unit": rl["unit"], "frac": rl["frac"],
+                     "traffic": rl["traffic"],
+                     "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json: sustained bf16 for "
+                                    "tensor-bound kernels, copy bandwidth for HBM-bound ones)"},
+        "kernel_rooflines": {k: _kernel_roofline(k, b, w, per_kernel[k], peaks, traffic.get(k))
+                             for k, (b, w) in names.items()},
+        "step_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": ms_per_step * 1e3,
+                          "frac": t_roof / (ms_per_step / 1e3), "flops": wk["flops"],
+                          "bytes": wk["bytes"]},
+        "kernels_ms_per_step": {k: v[0] / max(v[1], 1) for k, v in per_kernel.items()},
+        "gpu_launches": launches,
+        "device_error_word": err,
+        "burst": {"value": tokens / (burst_ms / 1e3), "ms_per_step": burst_ms / args.steps,
+                  "note": "the same K steps right after the warm-up, before the power "
+                          "controller reacts; value and rooflines above are the steady state"},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "clocks": clocks,
+    }
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -343,51 +389,9 @@ def run_ours(args):
 
     result = None
     if rank == 0:
-        peaks = _peaks()
-        wk = _work(inp)
-        ms_per_step = total_ms / args.steps
-        tokens = T * ws * args.steps
-        value = tokens / (total_ms / 1e3)
-        # dominant kernel by measured share
-        names = {"qkv_rope_scatter": ("tensor", wk["qkv_flops"]), "attention": ("hbm", wk["attn_bytes"])}
-        dom = max(names, key=lambda k: per_kernel[k][0])
-        ms_k, n_k = per_kernel[dom]
-        avg_s = ms_k / max(n_k, 1) / 1e3
-        bound, work = names[dom]
-        if bound == "tensor":
-            achieved = work / avg_s / 1e12
-            peak = peaks["bf16_tflops_sustained"]
-            unit = "TFLOP/s"
-        else:
-            achieved = work / avg_s / 1e9
-            peak = peaks["hbm_gbs"]
-            unit = "GB/s"
-        t_roof = max(wk["flops"] / (peaks["bf16_tflops_sustained"] * 1e12),
-                     wk["bytes"] / (peaks["hbm_gbs"] * 1e9))
-        traffic = _dram_traffic(args.workload)
-        result = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": inp.dtype, "data": "synthetic",
-            "config": _step_config(args.workload, inp, ws),
-            "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                         "frac": achieved / peak, "traffic": traffic.get(dom),
-                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json: sustained bf16 for "
-                                        "tensor-bound kernels, copy bandwidth for HBM-bound ones)"},
-            "kernel_rooflines": {k: _kernel_roofline(k, b, w, per_kernel[k], peaks, traffic.get(k))
-                                 for k, (b, w) in names.items()},
-            "step_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": ms_per_step * 1e3,
-                              "frac": t_roof / (ms_per_step / 1e3), "flops": wk["flops"], "bytes": wk["bytes"]},
-            "kernels_ms_per_step": {k: v[0] / max(v[1], 1) for k, v in per_kernel.items()},
-            "gpu_launches": launches,
-            "device_error_word": err,
-            "burst": {"value": tokens / (burst_ms / 1e3), "ms_per_step": burst_ms / args.steps,
-                      "note": "the same K steps right after the warm-up, before the power "
-                              "controller reacts; value and rooflines above are the steady state"},
-            "e2e": {"value": T * ws * args.steps / (e2e_ms / 1e3), "unit": UNIT,
-                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
-            "clocks": clk.summary(),
-        }
+        result = _step_result(args, inp, ws, total_ms=total_ms, burst_ms=burst_ms,
+                              per_kernel=per_kernel, launches=launches, err=err, e2e_ms=e2e_ms,
+                              h2d=h2d, d2h=d2h, clocks=clk.summary())
         # the oracle's timing is a single-GPU line's context: rank 0 at N = 1 only
         result["cpu_baseline"] = (cpu_baseline(inp, budget_s=args.cpu_budget)
                                   if args.cpu_budget > 0 and ws == 1 else None)

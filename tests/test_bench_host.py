@@ -92,3 +92,38 @@ def _tiny():
     from kv_cache_attention_qkv_b200 import workloads
 
     return workloads.generate("tiny_fp32")
+
+
+def test_step_result_line_follows_the_contract():
+    """The JSON line a step run prints, from made-up measurements: every key of
+    the contract, and the numbers derived from the timings as stated."""
+    import argparse
+
+    from kv_cache_attention_qkv_b200 import workloads
+
+    inp = workloads.generate("tiny_fp32")
+    args = argparse.Namespace(steps=10, warmup=3, workload="tiny_fp32")
+    per_kernel = {"prep": (0.1, 10), "qkv_rope_scatter": (3.0, 10), "attention": (2.0, 10),
+                  "importance_finalize": (0.05, 10), "topk": (0.1, 10)}
+    clocks = {"sm_mhz": 1600.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    r = bench._step_result(args, inp, 2, total_ms=5.0, burst_ms=4.0, per_kernel=per_kernel,
+                           launches=50, err=0, e2e_ms=8.0, h2d=1000, d2h=2000, clocks=clocks)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "roofline",
+                "e2e", "gpu_launches", "clocks"):
+        assert key in r, key
+    T = inp.total_q
+    assert r["value"] == pytest.approx(T * 2 * 10 / 5e-3)        # all ranks' tokens / max time
+    assert r["ms_per_step"] == pytest.approx(0.5) and r["n_gpus"] == 2
+    assert r["burst"]["value"] == pytest.approx(T * 2 * 10 / 4e-3)
+    assert r["e2e"] == {"value": pytest.approx(T * 2 * 10 / 8e-3), "unit": r["unit"],
+                        "h2d_bytes_per_step": 1000, "d2h_bytes_per_step": 2000}
+    rl = r["roofline"]
+    assert rl["kernel"] == "qkv_rope_scatter" and rl["bound"] == "tensor"  # the larger share
+    wk = bench._work(inp)
+    assert rl["achieved"] == pytest.approx(wk["qkv_flops"] / 0.3e-3 / 1e12)  # 0.3 ms per launch
+    assert rl["frac"] == pytest.approx(rl["achieved"] / rl["peak"])
+    assert rl["peak"] == bench._peaks()["bf16_tflops_sustained"]
+    att = r["kernel_rooflines"]["attention"]
+    assert att["unit"] == "GB/s" and att["achieved"] == pytest.approx(wk["attn_bytes"] / 0.2e-3 / 1e9)
+    assert r["clocks"] is clocks and r["gpu_launches"] == 50 and r["higher_is_better"] is True
