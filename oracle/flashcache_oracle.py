@@ -138,6 +138,8 @@ def attend_sequence(q: np.ndarray, k_cache_b: np.ndarray, v_cache_b: np.ndarray)
     L = k_cache_b.shape[0]
     o = np.empty((n, H, d), np.float64)
     P = np.empty((H, n, L), np.float64)
+    if n == 0:  # no query rows: nothing attends (the cache may be empty too)
+        return o, P
     scale = 1.0 / np.sqrt(d)
     for h in range(H):
         s = (q[:, h, :] @ np.asarray(k_cache_b[:, h, :], np.float64).T) * scale

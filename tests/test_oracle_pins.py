@@ -364,3 +364,17 @@ def test_sweep_workload_recipe(name, B, beta, L):
     with pytest.raises(ValueError):
         workloads.parse_sweep("sweep_b1_m63_L768")
     assert workloads.parse_sweep("batch32_uniform") is None
+
+
+def test_sequence_without_query_rows_contributes_nothing():
+    # the importance sums over the step's query rows: with none it is an empty sum
+    rng = _rng(31)
+    H, d, D = 2, 8, 16
+    w = rng.standard_normal((3 * H * d, D))
+    for L in (0, 5):
+        kc, vc = rng.standard_normal((L, H, d)), rng.standard_normal((L, H, d))
+        r = oracle.step_sequence(np.zeros((0, D)), w, np.zeros(0, np.int64), kc, vc, H, d, 1e4, None)
+        assert r["out"].shape == (0, H, d)
+        assert r["importance"].shape == (L,) and (r["importance"] == 0).all()
+        np.testing.assert_array_equal(r["k_cache"], kc)
+        np.testing.assert_array_equal(r["v_cache"], vc)
