@@ -229,6 +229,32 @@ FC_API fc_status fc_get_error(fc_handle* h, int32_t* device_error_word);
  */
 FC_API fc_status fc_selftest_wait_timeout(fc_handle* h, void* stream, int limit_us);
 
+/*
+ * fc_last_step_work — how the attention work of the handle's last fc_step was
+ * split (waits for the stream of the last call):
+ *   items           work items, one per (sequence, head, query tile);
+ *   two_pass_items  items given to the two-pass attention kernel from the
+ *                   start: all of them when the step asked for importance (it
+ *                   needs every row's final normaliser before the column sums,
+ *                   so that kernel scans K twice), none otherwise (bf16 tensor-
+ *                   core path; 0 on the CUDA-core path);
+ *   handed_over     items of a step without importance that the one-pass
+ *                   kernel handed to the two-pass kernel because a score
+ *                   exceeded its row's reference (the maximum over the item's
+ *                   first key tile) by more than 64 in log2 units.
+ * Host pointers.  For tests and measurement tools.
+ */
+FC_API fc_status fc_last_step_work(fc_handle* h, int32_t* items, int32_t* two_pass_items,
+                                   int32_t* handed_over);
+
+/*
+ * fc_last_cuda_error — text of the last CUDA failure behind an FC_ERR_CUDA of
+ * fc_step on this handle: the kernel being launched and CUDA's error name and
+ * string ("no CUDA error recorded" if none).  The pointer stays valid until
+ * the calling thread's next call.
+ */
+FC_API const char* fc_last_cuda_error(const fc_handle* h);
+
 /* Number of kernels the last fc_step / fc_topk_tracked call enqueued (host). */
 FC_API int fc_last_launch_count(const fc_handle* h);
 
@@ -237,11 +263,15 @@ FC_API int fc_last_launch_count(const fc_handle* h);
  * fc_step / fc_topk_tracked record a CUDA event pair on its stream around each
  * kernel it launches (up to 4096 launches); fc_profile(h, 0) stops recording.
  * fc_profile_read waits for the recorded work, writes for each kernel slot
- * (0 prep, 1 qkv_rope_scatter, 2 attention, 3 importance_finalize, 4 topk) the
- * summed milliseconds to ms[slot] and the launch count to launches[slot]
- * (host arrays of FC_PROFILE_SLOTS entries), and clears the record.
+ * (0 prep, 1 qkv_rope_scatter, 2 attention (the two-pass attention kernel
+ * of the tensor-core path: every item of a step with importance, the items
+ * handed over in a step without), 3 importance_finalize, 4 topk,
+ * 5 attention_one_pass (the one-pass kernel of a tensor-core step without
+ * importance)) the summed milliseconds to ms[slot] and the launch count to
+ * launches[slot] (host arrays of FC_PROFILE_SLOTS entries), and clears the
+ * record.
  */
-#define FC_PROFILE_SLOTS 5
+#define FC_PROFILE_SLOTS 6
 FC_API fc_status fc_profile(fc_handle* h, int enable);
 FC_API fc_status fc_profile_read(fc_handle* h, float* ms, int* launches);
 
@@ -262,16 +292,22 @@ FC_API fc_status fc_profile_read(fc_handle* h, float* ms, int* launches);
  *   cu_seqlens_q/k dev, int32 [B+1], as for fc_step (sequences with ranges
  *                  outside [0, T) / [0, S) are skipped)
  *   k_cache, v_cache dev, [S, H, d], only read
- *   out            dev, [T, H, d];  importance  dev, float [S]
- * Limits: S <= FC_NOALLOC_MAX_KEYS, d <= 256, B and H <= 65535; larger sizes
- * return FC_ERR_UNSUPPORTED before anything is queued.
+ *   out            dev, [T, H, d];  importance  dev, float [S].  Rows of a
+ *                  sequence whose cache is empty (L_b = 0) get zeros: they
+ *                  have no key to attend.
+ * Limits: S <= FC_NOALLOC_MAX_KEYS, d <= 256, B and H <= 65535, and
+ * H * T < 2^23 (a key's importance, at most H * T, is summed in signed 2^-40
+ * fixed point); larger sizes return FC_ERR_UNSUPPORTED before anything is
+ * queued.
  * Its scratch (a fixed-point accumulator of FC_NOALLOC_MAX_KEYS + 32 int64,
  * 512 KiB) is a static array in the library's device image: every GPU that
  * loads the library holds it until the process exits, and every call shares
  * it.  Each call clears the part it uses on `stream` first; calls whose work
  * overlaps on the GPU (two streams, or two threads) race on it.  The first
- * call on a device looks up the array's device address (once per device);
- * make that first call before any stream capture.
+ * call in a CUDA context looks up the array's device address in that context
+ * (once per context: the device's primary context, or each context the
+ * caller makes current); make that first call before any stream capture.  Do
+ * not keep using the library in a process across cudaDeviceReset.
  */
 #define FC_NOALLOC_MAX_KEYS 65536
 FC_API fc_status fc_attention_noalloc(void* stream, int dtype, int batch, int n_heads,
@@ -408,6 +444,10 @@ FC_API fc_handle* fc_model_layer_handle(fc_model* m);
  *                  the generated span (window_start + W <= gen_end <= L_b).
  *   tokens, draft  dev, int32 [S] (one entry per cache row, -1 = none), in/out.
  *   n_accepted     dev, int32 [B], out: tokens accepted this iteration.
+ *   importance     dev, float [S] or NULL: when given, receives the draft
+ *                  view's importance summed over layers, the scores the
+ *                  reselection of step 4 ranked (a handle-owned buffer is used
+ *                  otherwise).
  * Device-side checks (positions, ids) set the layer handle's error word.
  */
 FC_API fc_status fc_decode_iteration(fc_model* m, void* stream, int batch,
@@ -416,7 +456,24 @@ FC_API fc_status fc_decode_iteration(fc_model* m, void* stream, int batch,
                                      const void* embed, int mask_id, int n_tracked, int window,
                                      int32_t* tracked, int32_t* window_start,
                                      const int32_t* gen_end, int32_t* tokens, int32_t* draft,
-                                     int32_t* n_accepted);
+                                     int32_t* n_accepted, float* importance);
+
+/*
+ * fc_model_lm_head — the last stage of fc_model_step on rows the caller
+ * supplies: the LM head over rows that are already final-normed
+ * (rms_norm(h) * g_final), then per row the top token, its softmax
+ * probability (the confidence) and the Flash-Verify acceptance
+ * confidence >= threshold (paper-digest page, Flash-Verify).  The logits are
+ * never written: the kernel keeps per 256-column tile the maximum, its index
+ * and the sum of exp(logit - maximum), and a second kernel merges the tiles.
+ *   rows           dev, [n_rows, D] bf16, 16-byte aligned.
+ *   n_rows         1 <= n_rows <= max_head_rows of the model's config.
+ *   token, confidence, accept   dev, as for fc_model_step.
+ * Uses the model's LM-head statistics buffer: not concurrent with another
+ * call on the same model.
+ */
+FC_API fc_status fc_model_lm_head(fc_model* m, void* stream, const void* rows, int n_rows,
+                                  int32_t* token, float* confidence, uint8_t* accept);
 
 /* Release the model, its layer handle and workspace (NULL is a no-op). */
 FC_API void fc_model_destroy(fc_model* m);

@@ -26,8 +26,10 @@ EXPORTED = ("fc_create", "fc_step", "fc_topk_tracked", "fc_step_host", "fc_host_
             "fc_get_error", "fc_last_launch_count", "fc_profile", "fc_profile_read",
             "fc_attention_noalloc", "fc_selftest_wait_timeout", "fc_destroy", "fc_status_str",
             "fc_model_create", "fc_model_step", "fc_model_layer_handle", "fc_model_destroy",
-            "fc_decode_iteration")
-PROFILE_SLOTS = ("prep", "qkv_rope_scatter", "attention", "importance_finalize", "topk")
+            "fc_decode_iteration", "fc_model_lm_head", "fc_last_step_work",
+            "fc_last_cuda_error")
+PROFILE_SLOTS = ("prep", "qkv_rope_scatter", "attention", "importance_finalize", "topk",
+                 "attention_one_pass")
 
 
 class FlashCacheError(RuntimeError):
@@ -81,6 +83,10 @@ def load_library(path: Optional[str] = None):
     lib.fc_step_host.restype = c_int
     lib.fc_host_sync.argtypes = [vp, vp]
     lib.fc_host_sync.restype = c_int
+    lib.fc_last_cuda_error.argtypes = [vp]
+    lib.fc_last_cuda_error.restype = ctypes.c_char_p
+    lib.fc_last_step_work.argtypes = [vp, i32p, i32p, i32p]
+    lib.fc_last_step_work.restype = c_int
     lib.fc_get_error.argtypes = [vp, i32p]
     lib.fc_get_error.restype = c_int
     lib.fc_last_launch_count.argtypes = [vp]
@@ -107,8 +113,10 @@ def load_library(path: Optional[str] = None):
     lib.fc_model_destroy.argtypes = [vp]
     lib.fc_model_destroy.restype = None
     lib.fc_decode_iteration.argtypes = [vp, vp, c_int, vp, c_int, vp, vp, vp, c_int, c_int, c_int,
-                                        vp, vp, vp, vp, vp, vp]
+                                        vp, vp, vp, vp, vp, vp, vp]
     lib.fc_decode_iteration.restype = c_int
+    lib.fc_model_lm_head.argtypes = [vp, vp, vp, c_int, vp, vp, vp]
+    lib.fc_model_lm_head.restype = c_int
     lib.fc_status_str.argtypes = [c_int]
     lib.fc_status_str.restype = ctypes.c_char_p
     if path is None:
@@ -187,7 +195,10 @@ class FlashCache:
                               _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), T, S, _ptr(k_cache),
                               _ptr(v_cache), _ptr(out), _ptr(importance), int(bool(accumulate)))
         if st != 0:
-            raise FlashCacheError(st, "fc_step")
+            what = "fc_step"
+            if st == -3:
+                what += " (" + self.lib.fc_last_cuda_error(self._h).decode() + ")"
+            raise FlashCacheError(st, what)
 
     def topk_tracked(self, importance, cu_seqlens_k, cand_lo, cand_hi, k: int, tracked,
                      k_per_seq=None, stream=None) -> None:
@@ -252,6 +263,15 @@ class FlashCache:
         if st not in (0, -5, -6):
             raise FlashCacheError(st, "fc_get_error")
         return int(w.value)
+
+    def last_step_work(self):
+        """(work items, items of the two-pass kernel, items handed over to it) of
+        the last step; waits for the last stream used."""
+        a, b, c = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int32(0)
+        st = self.lib.fc_last_step_work(self._h, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c))
+        if st != 0:
+            raise FlashCacheError(st, "fc_last_step_work")
+        return int(a.value), int(b.value), int(c.value)
 
     def profile(self, enable: bool) -> None:
         """Record a CUDA event pair around every later kernel launch (or stop)."""
@@ -354,9 +374,13 @@ class FlashCacheModel:
 
     def decode_iteration(self, cu_seqlens_k, k_caches, v_caches, embed, mask_id: int, tracked,
                          window_start, gen_end, tokens, draft, n_accepted, window: int,
-                         stream=None) -> None:
+                         importance=None, stream=None) -> None:
         """Enqueue fc_decode_iteration; tracked is int32 [B, K], the state arrays are
-        int32 device tensors updated in place."""
+        int32 device tensors updated in place; importance (float [S] or None)
+        receives the draft view's importance the reselection ranked."""
+        if importance is not None and (importance.dtype != torch.float32 or not importance.is_cuda
+                                       or not importance.is_contiguous()):
+            raise FlashCacheError(-1, "importance must be a contiguous float32 CUDA tensor")
         B, K = tracked.shape
         kp = (ctypes.c_void_p * self.n_layers)(*[t.data_ptr() for t in k_caches])
         vp_ = (ctypes.c_void_p * self.n_layers)(*[t.data_ptr() for t in v_caches])
@@ -364,9 +388,23 @@ class FlashCacheModel:
                                           k_caches[0].shape[0], kp, vp_, _ptr(embed), int(mask_id),
                                           int(K), int(window), _ptr(tracked), _ptr(window_start),
                                           _ptr(gen_end), _ptr(tokens), _ptr(draft),
-                                          _ptr(n_accepted))
+                                          _ptr(n_accepted), _ptr(importance))
         if st != 0:
             raise FlashCacheError(st, "fc_decode_iteration")
+
+    def lm_head(self, rows, token, confidence, accept, stream=None) -> None:
+        """Enqueue fc_model_lm_head on final-normed bf16 rows [R, D]."""
+        if rows.dtype != torch.bfloat16 or not rows.is_cuda or not rows.is_contiguous() or \
+                rows.dim() != 2 or rows.shape[1] != self.hidden:
+            raise FlashCacheError(-1, "rows must be a contiguous bfloat16 CUDA tensor [R, hidden]")
+        R = rows.shape[0]
+        for t, dt in ((token, torch.int32), (confidence, torch.float32), (accept, torch.uint8)):
+            if t.dtype != dt or not t.is_cuda or not t.is_contiguous() or t.numel() < R:
+                raise FlashCacheError(-1, "token/confidence/accept: int32/float32/uint8 CUDA [R]")
+        st = self.lib.fc_model_lm_head(self._m, _stream_handle(stream), _ptr(rows), int(R),
+                                       _ptr(token), _ptr(confidence), _ptr(accept))
+        if st != 0:
+            raise FlashCacheError(st, "fc_model_lm_head")
 
     def get_error(self) -> int:
         """Wait for the last stream used and return (and clear) the device error word."""

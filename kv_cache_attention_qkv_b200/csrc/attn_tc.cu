@@ -8,9 +8,12 @@
 // one launch through block scheduling (infernews post "Flash-dLLM: IO-aware KV
 // caching and parallel decoding", Flash-Cache paragraph).
 //
-// One work item = (sequence b, head h, 128-row query tile).  The importance
-// needs the final softmax normalisation of every row before columns are
-// summed, so the cache is scanned twice:
+// One work item = (sequence b, head h, 128-row query tile).  This kernel takes
+// every item of a step that asks for importance, and in a step that does not,
+// the items the one-pass kernel (attn_onepass.cu) handed over because a score
+// left its safe exponent band.  The importance needs the final softmax
+// normalisation of every row before columns are summed, so the cache is
+// scanned twice:
 //   pass 1: S = Q K^T per 128-key tile, row max m and sum l;
 //   pass 2: S = Q K^T again, P = 2^(S - m - log2 l) (final probabilities),
 //           O += P V on the tensor cores, column sums of P in registers.
@@ -77,7 +80,9 @@ constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, 128, 0, 1);  // P V, V MN
 
 struct AttnParams {
   int H, max_T;
-  const WorkItem* items;
+  const WorkItem* items;     // the work list: its first sched[2] items come here
+  const WorkItem* items_fb;  // then the sched[3] items the one-pass kernel handed over
+  int max_fb;
   const int32_t* sched;
   const int32_t* cu_q;
   const int32_t* cu_k;
@@ -103,19 +108,29 @@ struct Item {
   int b, qt, h, q0, nrows, k0, L, ntiles;
 };
 
-__device__ __forceinline__ Item load_item(const AttnParams& p, int it) {
-  const WorkItem w = p.items[it];
+__device__ __forceinline__ Item to_item(const WorkItem& w) {
   Item r;
   r.b = w.seq;
   r.qt = w.tile_head >> 8;
   r.h = w.tile_head & 0xFF;
-  r.q0 = p.cu_q[r.b];
-  const int n = p.cu_q[r.b + 1] - r.q0;
-  r.nrows = min(QT, n - r.qt * QT);
-  r.k0 = p.cu_k[r.b];
-  r.L = p.cu_k[r.b + 1] - r.k0;
+  r.q0 = w.q0;
+  r.nrows = w.nrows;
+  r.k0 = w.k0;
+  r.L = w.L;
   r.ntiles = (r.L + KT - 1) / KT;
   return r;
+}
+
+// Address of item `it` of this kernel's list: the long items, then the
+// handed-over ones.
+__device__ __forceinline__ const WorkItem* item_ptr(const AttnParams& p, int n_long, int it) {
+  return it < n_long ? p.items + it : p.items_fb + (it - n_long);
+}
+
+__device__ __forceinline__ WorkItem fetch_item(const AttnParams& p, int n_long, int n, int it) {
+  WorkItem w = {};
+  if (it < n) w = *item_ptr(p, n_long, it);
+  return w;
 }
 
 // Tiled 3-D TMA load with an L2 eviction-priority policy (createpolicy).
@@ -200,7 +215,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   bool failed = false;
   // the work list, Q and the refreshed cache come from the preceding kernels
   ptx::griddep_wait();
-  const int n_items = p.sched[0];
+  const int n_long = p.sched[2];
+  const int n_items = n_long + min(p.sched[3], p.max_fb);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -224,8 +240,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         ++prod;
         return true;
       };
+      // the next item's record is fetched while this one runs
+      WorkItem wnext = fetch_item(p, n_long, n_items, blockIdx.x);
       for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
-        const Item t = load_item(p, it);
+        const Item t = to_item(wnext);
+        wnext = fetch_item(p, n_long, n_items, it + gridDim.x);
         if (!ptx::mbar_wait(bar(bars->qfree), (ic & 1u) ^ 1u, abort_flag)) {
           failed = true;
           break;
@@ -306,8 +325,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         ptx::mma_commit(bar(bars->empty[idx % SLOTS]));
         return true;
       };
+      // the next item's record is fetched while this one runs
+      WorkItem wnext = fetch_item(p, n_long, n_items, blockIdx.x);
       for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
-        const Item t = load_item(p, it);
+        const Item t = to_item(wnext);
+        wnext = fetch_item(p, n_long, n_items, it + gridDim.x);
         if (!ptx::mbar_wait(bar(bars->qfull), ic & 1u, abort_flag)) {
           failed = true;
           break;
@@ -408,8 +430,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       return v[0];
     };
 
+    // the next item's record, field `lane` in lane `lane` (one register)
+    auto fetch_field = [&](int it) -> int {
+      return (lane < 6 && it < n_items)
+                 ? __ldg(reinterpret_cast<const int*>(item_ptr(p, n_long, it)) + lane)
+                 : 0;
+    };
+    int fnext = fetch_field(blockIdx.x);
     for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
-      const Item t = load_item(p, it);
+      WorkItem wcur;
+      wcur.seq = __shfl_sync(0xffffffffu, fnext, 0);
+      wcur.tile_head = __shfl_sync(0xffffffffu, fnext, 1);
+      wcur.q0 = __shfl_sync(0xffffffffu, fnext, 2);
+      wcur.nrows = __shfl_sync(0xffffffffu, fnext, 3);
+      wcur.k0 = __shfl_sync(0xffffffffu, fnext, 4);
+      wcur.L = __shfl_sync(0xffffffffu, fnext, 5);
+      const Item t = to_item(wcur);
+      fnext = fetch_field(it + gridDim.x);
       uint32_t sv[64];
       // ---- pass 1: max and normaliser over this warp's tiles and column half
       float m = -INFINITY, l = 0.f;
@@ -591,6 +628,8 @@ cudaError_t launch_attn_tc(const fc_handle* h, cudaStream_t st, const StepShape&
   p.H = s.H;
   p.max_T = h->cfg.max_total_q;
   p.items = h->ws.items;
+  p.items_fb = h->ws.items_fb;
+  p.max_fb = h->ws.max_items;
   p.sched = h->ws.sched;
   p.cu_q = cu_q;
   p.cu_k = cu_k;

@@ -168,7 +168,8 @@ fc_status fc_decode_iteration(fc_model* m, void* stream, int batch, const int32_
                               int total_k, void* const* k_caches, void* const* v_caches,
                               const void* embed, int mask_id, int n_tracked, int window,
                               int32_t* tracked, int32_t* window_start, const int32_t* gen_end,
-                              int32_t* tokens, int32_t* draft, int32_t* n_accepted) {
+                              int32_t* tokens, int32_t* draft, int32_t* n_accepted,
+                              float* importance_out) {
   if (!m || batch < 1 || n_tracked < 0 || window < 1 || !cu_seqlens_k || !embed || !tracked ||
       !window_start || !gen_end || !tokens || !draft || !n_accepted || !k_caches || !v_caches)
     return FC_ERR_INVALID_ARG;
@@ -176,7 +177,8 @@ fc_status fc_decode_iteration(fc_model* m, void* stream, int batch, const int32_
   const int T = batch * (n_tracked + window);
   if (mask_id < 0 || mask_id >= V || batch > fc::model_max_batch(m) ||
       T > fc::model_max_total_q(m) || batch * window > fc::model_max_head_rows(m) ||
-      n_tracked > fc::model_max_topk(m) || ((uintptr_t)embed & 15u))
+      n_tracked > fc::model_max_topk(m) || ((uintptr_t)embed & 15u) ||
+      (importance_out && ((uintptr_t)importance_out & 3u)))
     return FC_ERR_INVALID_ARG;
   fc_handle* h = fc::model_layer(m);
   if (cudaSetDevice(h->device) != cudaSuccess) return FC_ERR_CUDA;
@@ -204,7 +206,8 @@ fc_status fc_decode_iteration(fc_model* m, void* stream, int batch, const int32_
   int32_t *tok_m = (int32_t*)ws_slots[7], *tok_d = (int32_t*)ws_slots[8];
   float *conf_m = (float*)ws_slots[9], *conf_d = (float*)ws_slots[10];
   uint8_t *acc_m = (uint8_t*)ws_slots[11], *acc_d = (uint8_t*)ws_slots[12];
-  float* importance = (float*)ws_slots[13];
+  // the draft view's importance: the caller's buffer when given, else the workspace's
+  float* importance = importance_out ? importance_out : (float*)ws_slots[13];
   const int32_t* cand_lo = (const int32_t*)ws_slots[14];
   int launches = 0;
   if (fc::launch_pdl(fc::decode_query_kernel, dim3(batch), dim3(128), 0, st, batch, n_tracked,

@@ -63,6 +63,14 @@ struct ProfScope {
   }
 };
 
+// Record a failed CUDA call of a step (slot: the kernel being launched, or -1)
+// and return FC_ERR_CUDA.
+fc_status cuda_fail(fc_handle* h, int slot, cudaError_t e) {
+  h->last_cuda_err = e;
+  h->last_cuda_slot = slot;
+  return FC_ERR_CUDA;
+}
+
 }  // namespace
 
 namespace fc {
@@ -136,8 +144,8 @@ static fc_status validate_config(const fc_config* c) {
 
 static void free_workspace(fc_handle* h) {
   fc::Workspace& w = h->ws;
-  void* ptrs[] = {w.q_buf, w.row_dst, w.imp_acc,  w.items,
-                  w.sched, w.err,     w.rope_cos, w.rope_sin};
+  void* ptrs[] = {w.q_buf, w.row_dst,  w.imp_acc,  w.items,   w.sched,
+                  w.err,   w.rope_cos, w.rope_sin, w.items_fb};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   w = fc::Workspace{};
@@ -185,6 +193,8 @@ fc_status fc_create(const fc_config* cfg, const void* w_qkv, fc_handle** out) {
             cudaMalloc(&w.err, sizeof(int32_t)) == cudaSuccess &&
             cudaMalloc(&w.rope_cos, (size_t)cfg->max_pos * half * sizeof(float)) == cudaSuccess &&
             cudaMalloc(&w.rope_sin, (size_t)cfg->max_pos * half * sizeof(float)) == cudaSuccess;
+  if (ok && h->tc_attn)
+    ok = cudaMalloc(&w.items_fb, (size_t)w.max_items * sizeof(fc::WorkItem)) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     free_workspace(h);
@@ -271,44 +281,62 @@ fc_status fc::step_impl(fc_handle* h, const CUtensorMap* tm_w, void* stream, int
   cudaError_t e;
   {
     ProfScope ps(h, st, 0);
+    // tensor-core path: with importance every item goes to the two-pass
+    // kernel (long_tiles 0), without it to the one-pass kernel
     e = fc::launch_prep(h, st, s, q_pos, cu_seqlens_q, cu_seqlens_k,
-                        h->tc_attn ? fc::kTcQTile : fc::kSimtQTile);
+                        h->tc_attn ? fc::kTcQTile : fc::kSimtQTile,
+                        (h->tc_attn && want_imp) ? 0 : 0x7fffffff);
   }
-  if (e != cudaSuccess) return FC_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(h, 0, e);
   h->last_launches++;
   if (h->tc_gemm) {
     CUtensorMap tm_x;
     if (!fc::encode_bf16_2d(&tm_x, x, (uint64_t)total_q, (uint64_t)c.hidden,
                             (uint64_t)c.hidden * 2, fc::kQkvXBoxRows, 64))
-      return FC_ERR_CUDA;
+      return cuda_fail(h, -1, cudaErrorInvalidValue);
     ProfScope ps(h, st, 1);
     e = fc::launch_qkv_tc(h, st, s, tm_x, *tm_w, q_pos, k_cache, v_cache);
   } else {
     ProfScope ps(h, st, 1);
     e = fc::launch_qkv_simt(h, st, s, x, q_pos, k_cache, v_cache);
   }
-  if (e != cudaSuccess) return FC_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(h, 1, e);
   h->last_launches++;
   if (h->tc_attn) {
     CUtensorMap tm_k, tm_v;
     if (!fc::encode_kv_3d(&tm_k, k_cache, total_k, c.n_heads) ||
         !fc::encode_kv_3d(&tm_v, v_cache, total_k, c.n_heads))
-      return FC_ERR_CUDA;
-    ProfScope ps(h, st, 2);
-    e = fc::launch_attn_tc(h, st, s, tm_k, tm_v, cu_seqlens_q, cu_seqlens_k, out, want_imp);
+      return cuda_fail(h, -1, cudaErrorInvalidValue);
+    if (want_imp) {
+      // the importance needs every row's final normaliser: two scans of K
+      ProfScope ps(h, st, 2);
+      e = fc::launch_attn_tc(h, st, s, tm_k, tm_v, cu_seqlens_q, cu_seqlens_k, out, true);
+      if (e != cudaSuccess) return cuda_fail(h, 2, e);
+    } else {
+      {
+        ProfScope ps(h, st, 5);
+        e = fc::launch_attn_onepass(h, st, tm_k, tm_v, cu_seqlens_q, cu_seqlens_k, out);
+      }
+      if (e != cudaSuccess) return cuda_fail(h, 5, e);
+      h->last_launches++;
+      // the items the one-pass kernel handed over (usually none)
+      ProfScope ps(h, st, 2);
+      e = fc::launch_attn_tc(h, st, s, tm_k, tm_v, cu_seqlens_q, cu_seqlens_k, out, false);
+      if (e != cudaSuccess) return cuda_fail(h, 2, e);
+    }
   } else {
     ProfScope ps(h, st, 2);
     e = fc::launch_attn_simt(h, st, s, cu_seqlens_q, cu_seqlens_k, k_cache, v_cache, out,
                              want_imp);
+    if (e != cudaSuccess) return cuda_fail(h, 2, e);
   }
-  if (e != cudaSuccess) return FC_ERR_CUDA;
   h->last_launches++;
   if (want_imp) {
     {
       ProfScope ps(h, st, 3);
       e = fc::launch_importance_finalize(h, st, total_k, importance, accumulate);
     }
-    if (e != cudaSuccess) return FC_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(h, 3, e);
     h->last_launches++;
   }
   return FC_OK;
@@ -342,6 +370,20 @@ fc_status fc_topk_tracked(fc_handle* h, void* stream, int batch, int total_k,
   return FC_OK;
 }
 
+fc_status fc_last_step_work(fc_handle* h, int32_t* items, int32_t* two_pass_items,
+                            int32_t* handed_over) {
+  if (!h || !items || !two_pass_items || !handed_over) return FC_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return FC_ERR_CUDA;
+  if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return FC_ERR_CUDA;
+  int32_t sc[4] = {0, 0, 0, 0};
+  if (cudaMemcpy(sc, h->ws.sched, sizeof(sc), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return FC_ERR_CUDA;
+  *items = sc[0];
+  *two_pass_items = h->tc_attn ? sc[2] : 0;
+  *handed_over = h->tc_attn ? sc[3] : 0;
+  return FC_OK;
+}
+
 fc_status fc_get_error(fc_handle* h, int32_t* device_error_word) {
   if (!h || !device_error_word) return FC_ERR_INVALID_ARG;
   if (cudaSetDevice(h->device) != cudaSuccess) return FC_ERR_CUDA;
@@ -356,6 +398,18 @@ fc_status fc_get_error(fc_handle* h, int32_t* device_error_word) {
 }
 
 int fc_last_launch_count(const fc_handle* h) { return h ? h->last_launches : 0; }
+
+const char* fc_last_cuda_error(const fc_handle* h) {
+  static const char* const kSlot[] = {"prep", "qkv_rope_scatter", "attention",
+                                      "importance_finalize", "topk", "attention_one_pass"};
+  static thread_local char buf[256];
+  if (!h || h->last_cuda_err == cudaSuccess) return "no CUDA error recorded";
+  snprintf(buf, sizeof(buf), "%s: %s (%s)",
+           h->last_cuda_slot >= 0 && h->last_cuda_slot < 6 ? kSlot[h->last_cuda_slot]
+                                                           : "host call",
+           cudaGetErrorName(h->last_cuda_err), cudaGetErrorString(h->last_cuda_err));
+  return buf;
+}
 
 fc_status fc_selftest_wait_timeout(fc_handle* h, void* stream, int limit_us) {
   if (!h || limit_us < 1 || limit_us > 2000000) return FC_ERR_INVALID_ARG;

@@ -45,10 +45,16 @@ struct GemmParams {
 constexpr double kImpScale = 1099511627776.0;  // 2^40
 constexpr double kImpInvScale = 1.0 / 1099511627776.0;
 
-// Work-list item: sequence, query tile, head.
-struct WorkItem {
+// Work-list item: sequence, query tile, head, and the item's ranges (written
+// by the prep kernel, so a kernel starts an item with one 32-byte load).
+struct __align__(16) WorkItem {
   int32_t seq;
   int32_t tile_head;  // (qtile << 8) | head
+  int32_t q0;         // first query row of the sequence
+  int32_t nrows;      // query rows of this tile
+  int32_t k0;         // first cache row of the sequence
+  int32_t L;          // cache rows of the sequence
+  int32_t pad[2];
 };
 
 struct Workspace {
@@ -56,7 +62,11 @@ struct Workspace {
   int32_t* row_dst = nullptr;             // [max_total_q] cache row of query row, or -1
   unsigned long long* imp_acc = nullptr;  // [max_total_k] fixed-point importance
   WorkItem* items = nullptr;              // attention work list
-  int32_t* sched = nullptr;               // [0] = item count, [1] = dynamic item counter
+  // [0] = item count, [1] = dynamic item counter (CUDA-core path),
+  // [2] = items for the two-pass kernel (the first ones of the list),
+  // [3] = items the one-pass kernel handed to the two-pass kernel
+  int32_t* sched = nullptr;
+  WorkItem* items_fb = nullptr;           // [max_items] those handed-over items
   int32_t* err = nullptr;                 // device error word
   float* rope_cos = nullptr;              // [max_pos, d/2]
   float* rope_sin = nullptr;              // [max_pos, d/2]
@@ -97,6 +107,10 @@ struct fc_handle {
   fc::Workspace ws;
   cudaStream_t last_stream = nullptr;
   int last_launches = 0;
+  // the last CUDA call of fc_step that failed: its error and the profile slot
+  // of the kernel being launched (-1: not a launch)
+  cudaError_t last_cuda_err = cudaSuccess;
+  int last_cuda_slot = -1;
   // optional per-kernel event timing (fc_profile)
   bool profiling = false;
   int prof_n = 0;
@@ -135,7 +149,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // ---- launchers (each returns the CUDA error of its launch) -----------------
 cudaError_t launch_prep(const fc_handle* h, cudaStream_t st, const StepShape& s,
                         const int32_t* q_pos, const int32_t* cu_q, const int32_t* cu_k,
-                        int qtile);
+                        int qtile, int long_tiles);
 cudaError_t launch_qkv_simt(const fc_handle* h, cudaStream_t st, const StepShape& s,
                             const void* x, const int32_t* q_pos, void* k_cache, void* v_cache);
 cudaError_t launch_attn_simt(const fc_handle* h, cudaStream_t st, const StepShape& s,
@@ -162,6 +176,10 @@ cudaError_t launch_attn_tc(const fc_handle* h, cudaStream_t st, const StepShape&
                            const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                            const int32_t* cu_q, const int32_t* cu_k, void* out,
                            bool want_importance);
+cudaError_t launch_attn_onepass(const fc_handle* h, cudaStream_t st, const CUtensorMap& tm_k,
+                                const CUtensorMap& tm_v, const int32_t* cu_q, const int32_t* cu_k,
+                                void* out);
+size_t attn_onepass_smem_bytes();
 cudaError_t launch_importance_finalize(const fc_handle* h, cudaStream_t st, int S,
                                        float* importance, int accumulate);
 cudaError_t launch_topk(const fc_handle* h, cudaStream_t st, int B, int S, const float* importance,

@@ -207,6 +207,32 @@ fc_status fc_model_step(fc_model* m, void* stream, int batch, const void* x, con
   return FC_OK;
 }
 
+fc_status fc_model_lm_head(fc_model* m, void* stream, const void* rows, int n_rows,
+                           int32_t* token, float* confidence, uint8_t* accept) {
+  if (!m || !al16(rows) || n_rows < 1 || n_rows > m->cfg.max_head_rows || !token || !confidence ||
+      !accept)
+    return FC_ERR_INVALID_ARG;
+  if (cudaSetDevice(m->layer->device) != cudaSuccess) return FC_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int D = m->cfg.layer.hidden;
+  CUtensorMap tm_rows;
+  if (!enc(&tm_rows, rows, (uint64_t)n_rows, (uint64_t)D)) return FC_ERR_CUDA;
+  fc::GemmParams p = {};
+  p.mode = fc::GEMM_LMHEAD;
+  p.M = n_rows;
+  p.N = m->cfg.vocab;
+  p.K = D;
+  p.partials = m->partials;
+  p.err = m->layer->ws.err;
+  if (fc::launch_gemm_tc(m->layer->num_sms, st, tm_rows, m->tm_lm, m->tm_lm, p) != cudaSuccess ||
+      fc::launch_lmhead_reduce(st, m->partials, n_rows, m->num_vn, m->cfg.threshold, token,
+                               confidence, accept) != cudaSuccess)
+    return FC_ERR_CUDA;
+  m->layer->last_stream = st;
+  m->layer->last_launches = 2;
+  return FC_OK;
+}
+
 void fc_model_destroy(fc_model* m) {
   if (!m) return;
   cudaSetDevice(m->layer->device);

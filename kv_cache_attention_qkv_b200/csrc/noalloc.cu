@@ -17,6 +17,7 @@
 // work; its last CTA converts the accumulator into `importance`.
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "fc_internal.h"
@@ -49,8 +50,9 @@ __device__ __forceinline__ __nv_bfloat16 st_f<__nv_bfloat16>(float v) {
   return __float2bfloat16_rn(v);
 }
 
-// grid = (ceil(T / 16), H, B); block = 128 threads (4 warps x 4 query rows).
-// acc[0 .. S) must be zero and acc[S] (the ticket) zero at launch.
+// grid = (X, H, B); block = 128 threads (4 warps x 4 query rows).  CTA
+// (x, h, b) takes the 16-row query tiles x, x + X, x + 2X, ... of sequence b
+// and head h.  acc[0 .. S) must be zero and acc[S] (the ticket) zero at launch.
 template <typename T>
 __global__ void __launch_bounds__(128) attn_noalloc_kernel(
     int B, int H, int d, int Ttot, int Stot, float qk_scale_log2, const T* __restrict__ q,
@@ -63,16 +65,20 @@ __global__ void __launch_bounds__(128) attn_noalloc_kernel(
   float* vs = ks + NA_KEYS * (d + 1);  // [32][d]
   float* cs = vs + NA_KEYS * d;        // [4][32]
   __shared__ bool last_cta;
-  unsigned int* ticket = reinterpret_cast<unsigned int*>(acc + Stot);
+  unsigned long long* ticket = acc + Stot;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qt = blockIdx.x, hh = blockIdx.y, b = blockIdx.z;
+  const int hh = blockIdx.y, b = blockIdx.z;
   const int q0 = cu_q[b], n = cu_q[b + 1] - q0, k0 = cu_k[b], L = cu_k[b + 1] - k0;
   const bool ok = q0 >= 0 && n >= 0 && q0 + n <= Ttot && k0 >= 0 && L >= 0 && k0 + L <= Stot;
-  const int rbeg = qt * NA_ROWS;
-  const int nrows = ok ? min(NA_ROWS, n - rbeg) : 0;
-
-  if (nrows > 0 && L > 0) {
+  for (int qt = blockIdx.x; ok && qt * NA_ROWS < n; qt += gridDim.x) {
+    const int rbeg = qt * NA_ROWS;
+    const int nrows = min(NA_ROWS, n - rbeg);
+    if (L == 0) {  // no key to attend: the rows' output is an empty sum, zero
+      for (int e = tid; e < nrows * d; e += 128)
+        out[((size_t)(q0 + rbeg + e / d) * H + hh) * d + e % d] = st_f<T>(0.f);
+      continue;
+    }
     for (int e = tid; e < NA_ROWS * d; e += 128) {
       const int rr = e / d, c = e % d;
       qs[e] = rr < nrows ? ld_f(q + ((size_t)(q0 + rbeg + rr) * H + hh) * d + c) * qk_scale_log2 : 0.f;
@@ -158,14 +164,16 @@ __global__ void __launch_bounds__(128) attn_noalloc_kernel(
         if (c < d) orow[c] = st_f<T>(o[a][t]);
       }
     }
+    __syncthreads();  // the shared tiles are reused by the next query tile
   }
 
   // the last CTA to finish turns the accumulator into floats
   __threadfence();
   __syncthreads();
   if (tid == 0) {
-    const unsigned int total = gridDim.x * gridDim.y * gridDim.z;
-    last_cta = atomicAdd(ticket, 1u) == total - 1;
+    const unsigned long long total =
+        (unsigned long long)gridDim.x * gridDim.y * gridDim.z;
+    last_cta = atomicAdd(ticket, 1ull) == total - 1ull;
   }
   __syncthreads();
   if (last_cta) {
@@ -175,23 +183,56 @@ __global__ void __launch_bounds__(128) attn_noalloc_kernel(
   }
 }
 
-std::mutex g_mu;
-void* g_scratch[64] = {nullptr};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
 
-// Device address of the scratch array on the current device, looked up once
-// per device (host code cannot use the array's name as a device address).
-void* scratch_address(int dev) {
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (dev < 0 || dev >= 64) return nullptr;
-  if (!g_scratch[dev]) {
+std::mutex g_mu;
+// (context, device address of the scratch in it), one entry per context seen
+constexpr int kMaxCtx = 64;
+CUcontext g_ctx[kMaxCtx] = {};
+void* g_scratch[kMaxCtx] = {};
+int g_nctx = 0;
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_acc) != cudaSuccess) {
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (CtxGetCurrentFn)p;
+  }
+  return fn;
+}
+
+// Device address of the scratch array in the current context, looked up the
+// first time a context calls (host code cannot use the array's name as a
+// device address).  Keyed by context, so a process that creates its own
+// contexts gets each one's copy of the array.
+void* scratch_address() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  CtxGetCurrentFn get = ctx_get_current();
+  CUcontext ctx = nullptr;
+  if (!get || get(&ctx) != CUDA_SUCCESS) return nullptr;
+  if (!ctx) {  // no context bound yet: the runtime's device, primary context
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess ||
+        get(&ctx) != CUDA_SUCCESS || !ctx) {
       cudaGetLastError();
       return nullptr;
     }
-    g_scratch[dev] = p;
   }
-  return g_scratch[dev];
+  for (int i = 0; i < g_nctx; ++i)
+    if (g_ctx[i] == ctx) return g_scratch[i];
+  if (g_nctx == kMaxCtx) return nullptr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_acc) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  g_ctx[g_nctx] = ctx;
+  g_scratch[g_nctx] = p;
+  ++g_nctx;
+  return p;
 }
 
 }  // namespace
@@ -206,18 +247,23 @@ extern "C" fc_status fc_attention_noalloc(void* stream, int dtype, int batch, in
       total_q < 0 || total_k < 0)
     return FC_ERR_INVALID_ARG;
   if (head_dim > NA_MAXD || total_k > FC_NOALLOC_MAX_KEYS) return FC_ERR_UNSUPPORTED;
+  // a key's importance is at most (heads x query rows); the signed 2^-40 fixed
+  // point accumulator holds sums below 2^23
+  if ((long long)n_heads * total_q >= (1ll << 23)) return FC_ERR_UNSUPPORTED;
   if (!cu_seqlens_q || !cu_seqlens_k || !importance) return FC_ERR_INVALID_ARG;
   if (total_q > 0 && (!q || !k_cache || !v_cache || !out)) return FC_ERR_INVALID_ARG;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return FC_ERR_CUDA;
-  unsigned long long* acc = static_cast<unsigned long long*>(scratch_address(dev));
+  unsigned long long* acc = static_cast<unsigned long long*>(scratch_address());
   if (!acc) return FC_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
   // accumulator of the keys in use and the ticket counter start at zero
   if (cudaMemsetAsync(acc, 0, ((size_t)total_k + 1) * sizeof(unsigned long long), st) != cudaSuccess)
     return FC_ERR_CUDA;
-  const int qtiles = total_q > 0 ? (total_q + NA_ROWS - 1) / NA_ROWS : 1;
-  dim3 grid(qtiles, n_heads, batch);
+  // query tiles per (sequence, head) CTA column: the batch's average tile
+  // count, so the grid holds about as many CTAs as there are tiles; a longer
+  // sequence's CTAs loop over its further tiles
+  const long long tiles = (total_q + NA_ROWS - 1) / NA_ROWS;
+  const int gx = (int)std::max(1ll, (tiles + batch - 1) / batch);
+  dim3 grid(gx, n_heads, batch);
   const int d = head_dim;
   const size_t smem = sizeof(float) * (NA_ROWS * d + NA_KEYS * (d + 1) + NA_KEYS * d + 4 * NA_KEYS);
   const float scale = (float)(1.4426950408889634 / sqrt((double)d));

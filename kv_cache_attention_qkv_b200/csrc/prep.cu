@@ -26,14 +26,18 @@ __device__ __forceinline__ bool seq_ok(const int32_t* cu_q, const int32_t* cu_k,
   return ok;
 }
 
-// Blocks 0..B-1: one sequence each.  Block B: the work list.
+// Blocks 0..B-1: one sequence each.  Block B: the work list.  Items of
+// sequences whose cache spans more than long_tiles 128-key tiles come first
+// (the list is ordered by cache length); sched[2] counts them: the two-pass
+// attention kernel takes those, the one-pass kernel the rest.
 __global__ void __launch_bounds__(512) prep_kernel(StepShape s, const int32_t* __restrict__ q_pos,
                                                    const int32_t* __restrict__ cu_q,
                                                    const int32_t* __restrict__ cu_k,
                                                    int32_t* __restrict__ row_dst,
                                                    WorkItem* __restrict__ items, int max_items,
                                                    int32_t* __restrict__ sched,
-                                                   int32_t* __restrict__ err, int qtile) {
+                                                   int32_t* __restrict__ err, int qtile,
+                                                   int long_tiles) {
   extern __shared__ uint32_t smem[];
   const int b = blockIdx.x;
   const int tid = threadIdx.x, nt = blockDim.x;
@@ -149,9 +153,21 @@ __global__ void __launch_bounds__(512) prep_kernel(StepShape s, const int32_t* _
       if (i < s.B) cnt[i] = carry + incl - v;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
+    __syncwarp();  // every lane's offsets are read below
     if (tid == 0) {
+      int n_long = carry;  // offset of the first sequence within long_tiles
+      for (int i = 0; i < s.B; ++i) {
+        if (!(key[i] >> 63)) break;
+        const int L = (int)((key[i] >> 32) & 0x7FFFFFFFull);
+        if ((L + 127) / 128 <= long_tiles) {
+          n_long = cnt[i];
+          break;
+        }
+      }
       sched[0] = min(carry, max_items);
       sched[1] = 0;
+      sched[2] = min(n_long, max_items);
+      sched[3] = 0;
     }
   }
   __syncthreads();
@@ -160,9 +176,11 @@ __global__ void __launch_bounds__(512) prep_kernel(StepShape s, const int32_t* _
     const int bq = sseq[i], nqt = snq[i];
     const int c = s.H * nqt;
     const int off = cnt[i];
+    const int q0 = cu_q[bq], n = cu_q[bq + 1] - q0, k0 = cu_k[bq], L = cu_k[bq + 1] - k0;
     for (int t = tid; t < c; t += nt) {
       const int hh = t / nqt, qt = t - hh * nqt;
-      if (off + t < max_items) items[off + t] = WorkItem{bq, (qt << 8) | hh};
+      if (off + t < max_items)
+        items[off + t] = WorkItem{bq, (qt << 8) | hh, q0, min(qtile, n - qt * qtile), k0, L, {0, 0}};
     }
   }
 }
@@ -179,7 +197,7 @@ size_t prep_smem_bytes(int max_pos, int max_batch) {
 
 cudaError_t launch_prep(const fc_handle* h, cudaStream_t st, const StepShape& s,
                         const int32_t* q_pos, const int32_t* cu_q, const int32_t* cu_k,
-                        int qtile) {
+                        int qtile, int long_tiles) {
   size_t smem = prep_smem_bytes(h->cfg.max_pos, h->cfg.max_batch);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -187,7 +205,8 @@ cudaError_t launch_prep(const fc_handle* h, cudaStream_t st, const StepShape& s,
     if (e != cudaSuccess) return e;
   }
   prep_kernel<<<s.B + 1, 512, smem, st>>>(s, q_pos, cu_q, cu_k, h->ws.row_dst, h->ws.items,
-                                           h->ws.max_items, h->ws.sched, h->ws.err, qtile);
+                                           h->ws.max_items, h->ws.sched, h->ws.err, qtile,
+                                           long_tiles);
   return cudaGetLastError();
 }
 

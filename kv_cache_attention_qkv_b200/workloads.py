@@ -17,6 +17,9 @@ Five workloads are defined, named by what they are:
                      hidden 256, 4 heads x 128, caches of 129..700 rows.
 * ``small_d64``      bf16 with head_dim 64 (the CUDA-core path): B=2, hidden
                      96, 3 heads x 64, caches of 200 and 333 rows.
+* ``small_longcache`` the small_varlen layer with caches of 2049, 2048, 700
+                     and 129 rows: ragged key tiles over the longest caches of
+                     the element-wise parity cases.
 
 Sweep points are named ``sweep_b<B>_m<beta>_L<L>``: the headline recipe with
 B sequences, a query of beta rows (beta/2 tracked + a beta/2-row window) and a
@@ -39,7 +42,7 @@ from typing import Dict, List, Optional
 import numpy as np
 
 WORKLOADS = ("tiny_fp32", "layer_b1", "batch32_uniform", "batch32_varlen", "small_varlen",
-             "small_d64")
+             "small_d64", "small_longcache")
 
 
 @dataclasses.dataclass
@@ -198,6 +201,16 @@ def generate(name: str, seed: Optional[int] = None, batch: Optional[int] = None)
         windows = [[16, 64][i % 2] for i in range(B)]
         budgets = [[40, 64][i % 2] for i in range(B)]
         starts = [[48, 256][i % 2] for i in range(B)]
+    elif name == "small_longcache":
+        dtype, D, H, d, theta, w_std = "bf16", 256, 4, 128, 5.0e5, 0.0625
+        B = batch or 4
+        lens = [[2049, 2048, 700, 129][i % 4] for i in range(B)]
+        windows = [[64, 16, 64, 16][i % 4] for i in range(B)]
+        budgets = [[80, 48, 100, 48][i % 4] for i in range(B)]
+        starts = []
+        for L, w, kb in zip(lens, windows, budgets):
+            first = -(-kb // w) * w
+            starts.append(int(first + w * rng.integers(0, (L - w - first) // w + 1)))
     else:  # small_varlen
         dtype, D, H, d, theta, w_std = "bf16", 256, 4, 128, 5.0e5, 0.0625
         B = batch or 3
@@ -248,6 +261,8 @@ def describe(name: str) -> Dict[str, object]:
                              cache="700,129,333", query="80+64, 48+16, 100+64"),
         "small_d64": dict(dtype="bf16", B=2, hidden=96, heads=3, head_dim=64,
                           cache="200,333", query="40+16, 64+64"),
+        "small_longcache": dict(dtype="bf16", B=4, hidden=256, heads=4, head_dim=128,
+                             cache="2049,2048,700,129", query="80+64, 48+16, 100+64, 48+16"),
     }
     return table[name]
 

@@ -155,13 +155,29 @@ def test_model_create_rejects_null_and_misaligned_weights(lib):
                                ctypes.byref(m)) == -1
 
 
+def test_noalloc_rejects_sizes_beyond_its_limits_before_any_cuda_call(lib):
+    """Sizes past the static scratch, or an importance sum that could leave its
+    fixed-point range (heads x query rows >= 2^23), are refused on the host."""
+    vp = ctypes.c_void_p(16)
+    bf16 = 0
+    assert lib.fc_attention_noalloc(None, bf16, 1, 1, 128, vp, vp, vp, 1, 65536 + 1, vp, vp, vp,
+                                    vp) == -2
+    assert lib.fc_attention_noalloc(None, bf16, 1, 128, 128, vp, vp, vp, 65536, 16, vp, vp, vp,
+                                    vp) == -2
+    assert lib.fc_attention_noalloc(None, bf16, 1, 1, 257, vp, vp, vp, 1, 16, vp, vp, vp, vp) == -2
+    assert lib.fc_attention_noalloc(None, 7, 1, 1, 128, vp, vp, vp, 1, 16, vp, vp, vp, vp) == -1
+    assert lib.fc_attention_noalloc(None, bf16, 1, 1, 128, vp, None, vp, 1, 16, vp, vp, vp,
+                                    vp) == -1
+
+
 def test_model_and_host_step_calls_on_null_handles_are_rejected(lib):
     vp = ctypes.c_void_p
     arr = (ctypes.c_void_p * 2)(16, 16)
     assert lib.fc_model_step(None, None, 1, vp(16), vp(16), vp(16), vp(16), 1, 1, arr, arr, None,
                              0, None, None, None, None, None) == -1
     assert lib.fc_decode_iteration(None, None, 1, vp(16), 1, arr, arr, vp(16), 0, 1, 1, vp(16),
-                                   vp(16), vp(16), vp(16), vp(16), vp(16)) == -1
+                                   vp(16), vp(16), vp(16), vp(16), vp(16), None) == -1
+    assert lib.fc_model_lm_head(None, None, vp(16), 1, vp(16), vp(16), vp(16)) == -1
     assert lib.fc_step_host(None, None, 1, vp(16), vp(16), vp(16), vp(16), 1, 1, vp(16), vp(16),
                             vp(16), vp(16), None, 1, vp(16), vp(16)) == -1
     assert lib.fc_host_sync(None, None) == -1

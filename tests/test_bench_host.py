@@ -127,3 +127,18 @@ def test_step_result_line_follows_the_contract():
     att = r["kernel_rooflines"]["attention"]
     assert att["unit"] == "GB/s" and att["achieved"] == pytest.approx(wk["attn_bytes"] / 0.2e-3 / 1e9)
     assert r["clocks"] is clocks and r["gpu_launches"] == 50 and r["higher_is_better"] is True
+    # the step against every peak variant, reproducible from the peaks file and
+    # the sampled clock
+    pk = bench._peaks()
+    st = r["step_roofline"]
+    scaled = pk["bf16_tflops_sustained"] * 1600.0 / pk["sustained_mhz"]
+    want = {"sustained": pk["bf16_tflops_sustained"], "burst": pk["bf16_tflops"],
+            "spec": bench.SPEC_BF16_TFLOPS, "sustained_clock_scaled": scaled}
+    for k, tf in want.items():
+        bw = bench.SPEC_HBM_GBS if k == "spec" else pk["hbm_gbs"]
+        t = max(wk["flops"] / (tf * 1e12), wk["bytes"] / (bw * 1e9))
+        assert st["variants"][k]["frac"] == pytest.approx(t / 0.5e-3), k
+    assert st["frac"] == st["variants"]["sustained"]["frac"]
+    assert st["judged_on"] == "sustained_clock_scaled"
+    assert rl["frac_vs"]["sustained_clock_scaled"] == pytest.approx(rl["achieved"] / scaled)
+    assert rl["frac_vs"]["spec"] == pytest.approx(rl["achieved"] / bench.SPEC_BF16_TFLOPS)

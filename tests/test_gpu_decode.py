@@ -4,6 +4,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from oracle import decode_oracle as do
 from kv_cache_attention_qkv_b200 import workloads
 import fc_testlib as tl
@@ -18,6 +19,10 @@ def _need_gpu(cuda_ok):
 
 def _f64(t):
     return t.float().cpu().numpy().astype(np.float64)
+
+
+# relative tolerance of a confidence (see the model-step parity test)
+CONF_TOL = 5e-2
 
 
 def _tok_ok(tok, logits, vocab):
@@ -55,16 +60,24 @@ def test_decode_iterations_follow_the_oracle(threshold, iters):
     st = {"tokens": i32(tokens), "draft": i32(np.full(mi.total_k, -1)), "tracked": i32(tracked),
           "ws": i32(prompt), "n_acc": i32(np.zeros(B))}
     gen_end, cu_k = i32(L), i32(mi.cu_seqlens_k)
+    imp_t = torch.full((mi.total_k,), float("nan"), device=dev)
     layers64 = [{k: _f64(v) for k, v in lw.items()} for lw in mi.layers]
     fn64, lm64, emb64 = _f64(mi.final_norm), _f64(mi.lm_head), _f64(mi.embed)
     for it in range(iters):
         before = {k: v.cpu().numpy() for k, v in st.items()}
         caches = ([_f64(t) for t in mi.k_caches], [_f64(t) for t in mi.v_caches])
         model.decode_iteration(cu_k, mi.k_caches, mi.v_caches, mi.embed, mask_id, st["tracked"],
-                               st["ws"], gen_end, st["tokens"], st["draft"], st["n_acc"], W)
+                               st["ws"], gen_end, st["tokens"], st["draft"], st["n_acc"], W,
+                               importance=imp_t)
         torch.cuda.synchronize()
         assert model.get_error() == 0, it
         after = {k: v.cpu().numpy() for k, v in st.items()}
+        imp_dev = imp_t.cpu().numpy().astype(np.float64)
+        # the reselection, bit for bit: the oracle's top-k over [0, ws) (ws as
+        # advanced) of the very importance the device ranked
+        want_tr = oracle.topk_tracked(imp_dev, mi.cu_seqlens_k, np.zeros(B, np.int32), after["ws"],
+                                      np.full(B, K, np.int32), K)
+        np.testing.assert_array_equal(after["tracked"], want_tr, err_msg=f"iteration {it}")
         for b in range(B):
             ks = slice(int(mi.cu_seqlens_k[b]), int(mi.cu_seqlens_k[b + 1]))
             ws0 = int(before["ws"][b])
@@ -83,10 +96,22 @@ def test_decode_iterations_follow_the_oracle(threshold, iters):
             if not und.any():
                 assert len(new) == 0, (it, b)  # the sequence's last window is done
             elif (conf_m[und] >= threshold).any():
-                assert new.tolist() == want.tolist(), (it, b)  # acceptance by threshold
+                # acceptance by threshold: the oracle's decision wherever the
+                # confidence is not within the tolerance of the threshold
+                clear = np.abs(conf_m - threshold) > CONF_TOL * threshold
+                sel = und & clear
+                assert np.array_equal(np.isin(np.nonzero(sel)[0], new), (conf_m >= threshold)[sel]), (it, b)
             else:
-                # at least one: the device's choice has (within 5e-2) the highest confidence
-                assert len(new) == 1 and conf_m[new[0]] >= conf_m[und].max() * (1 - 5e-2), (it, b)
+                # at least one: the oracle's choice (highest [MASK]-view confidence,
+                # lowest position on ties) wherever the best two undecided
+                # confidences are further apart than the tolerance; otherwise one
+                # of the positions within the tolerance of the best
+                assert len(new) == 1, (it, b)
+                cu_ = np.sort(conf_m[und])[::-1]
+                if len(cu_) == 1 or cu_[0] - cu_[1] > CONF_TOL * cu_[0]:
+                    assert new.tolist() == want.tolist(), (it, b, new, want)
+                else:
+                    assert conf_m[new[0]] >= cu_[0] * (1 - CONF_TOL), (it, b)
             for j in new:
                 assert _tok_ok(got_tok[win[j]], lg_m[j], mi.vocab), (it, b, j)
             # drafts of the still-undecided positions: the [MASK] view's predictions
@@ -95,15 +120,11 @@ def test_decode_iterations_follow_the_oracle(threshold, iters):
             assert after["ws"][b] == ref["ws"], (it, b)
             if threshold == 0.0 and ws0 + 2 * W <= L[b]:
                 assert after["ws"][b] == ws0 + W, (it, b)  # the window advanced
-            # tracked: K distinct positions of [0, ws), each within 2e-2 of the oracle's
-            # K-th largest importance there (the device's importance agrees with the
-            # oracle's to ~1e-2 here, and near-uniform attention makes many near-ties)
-            tr = after["tracked"][b]
-            hi = int(after["ws"][b])
-            imp = ref["importance"][:hi]
-            kth = np.sort(imp)[::-1][K - 1]
-            assert len(set(tr.tolist())) == K and tr.min() >= 0 and tr.max() < hi, (it, b)
-            assert (imp[tr] >= kth * (1 - 2e-2)).all(), (it, b, imp[tr].min(), kth)
+            # the importance the reselection ranked (the draft view's, summed over
+            # layers) against the oracle's, at the bf16 bar
+            # (the tracked set itself was checked bit for bit above)
+            tl.assert_close(imp_dev[ks], ref["importance"], 1e-2,
+                            f"iteration {it} seq {b} importance")
             # the caches keep the draft view's rows
             for l in range(mi.n_layers):
                 tl.assert_close(_f64(mi.k_caches[l][ks]), ref["k_caches"][l], 1e-2,

@@ -92,8 +92,36 @@ def compare_sequence(mi, got, ref, b, check_importance=True):
     for i, t in enumerate(tok):
         # a different token is accepted only when its logit ties the top one
         assert 0 <= t < mi.vocab and lg[i, t] >= lg[i].max() - 5e-3 * spread[i], (b, i, t)
+    # acceptance: the oracle's decision (confidence >= 0.9) on every row whose
+    # oracle confidence is not within the confidence tolerance of the threshold
     acc = got["accept"].cpu().numpy()[rows]
-    np.testing.assert_array_equal(acc, (conf >= 0.9).astype(np.uint8))
+    clear = np.abs(ref["confidence"] - 0.9) > 5e-2 * 0.9
+    np.testing.assert_array_equal(acc[clear], (ref["confidence"][clear] >= 0.9).astype(np.uint8),
+                                  err_msg=f"accept seq {b}")
+    assert set(np.unique(acc).tolist()) <= {0, 1}
+
+
+def check_lm_head_on_device_rows(mi, model, got):
+    """The LM-head kernel alone, fed the final norm of the device's own last
+    residual stream (rounded to bf16, the input the kernel sees inside the
+    model step), against the oracle's LM head on the same rows: the kernel's
+    own error, without the activations' drift through the layers."""
+    rows = mo.act_round(mo.rms_norm(_f64(got["h"])[mi.head_rows], _f64(mi.final_norm)), "bf16")
+    dev = mi.x_mask.device
+    R = len(mi.head_rows)
+    tok = torch.full((R,), -7, dtype=torch.int32, device=dev)
+    conf = torch.full((R,), float("nan"), device=dev)
+    acc = torch.full((R,), 7, dtype=torch.uint8, device=dev)
+    model.lm_head(torch.from_numpy(rows).to(dev, dtype=torch.bfloat16), tok, conf, acc)
+    torch.cuda.synchronize()
+    ref = mo.lm_head_confidence(rows, _f64(mi.lm_head))
+    np.testing.assert_allclose(conf.cpu().numpy(), ref["confidence"], rtol=1e-3,
+                               err_msg="LM head on the device's rows")
+    lg, tk = ref["logits"], tok.cpu().numpy()
+    spread = np.abs(lg).max(axis=1)
+    for i, t in enumerate(tk):
+        assert 0 <= t < mi.vocab and lg[i, t] >= lg[i].max() - 1e-4 * spread[i], (i, t)
+    np.testing.assert_array_equal(acc.cpu().numpy(), (conf.cpu().numpy() >= 0.9).astype(np.uint8))
 
 
 def test_model_small_full_parity():
@@ -114,6 +142,7 @@ def test_model_small_full_parity():
             for l in range(mi.n_layers):
                 tl.assert_close(_f64(kcs[l][ks]), ref["k"][l], 1e-2, f"{view} k cache layer {l}")
                 tl.assert_close(_f64(vcs[l][ks]), ref["v"][l], 1e-2, f"{view} v cache layer {l}")
+        check_lm_head_on_device_rows(mi, model, got)
         # importance sums to layers x heads x query rows
         imp = got["importance"].cpu().numpy().astype(np.float64)
         for b in range(mi.batch):

@@ -15,7 +15,8 @@ def _need_gpu(cuda_ok):
     return cuda_ok
 
 
-@pytest.mark.parametrize("name", ["tiny_fp32", "small_d64", "small_varlen", "layer_b1"])
+@pytest.mark.parametrize("name", ["tiny_fp32", "small_d64", "small_varlen", "layer_b1",
+                                  "small_longcache"])
 def test_full_parity(name):
     """Every output element of small workloads against the oracle."""
     inp = workloads.generate(name)
@@ -51,6 +52,96 @@ def test_full_size_sampled_parity(name, seqs):
         tot = imp[inp.seq_slice_k(b)].sum()
         assert abs(tot - inp.n_heads * n) <= 1e-3 * inp.n_heads * n, (b, tot)
     assert np.isfinite(gpu["out"]).all()
+
+
+def test_attention_work_split():
+    """A step with importance gives every item to the two-pass kernel (the column
+    sums need each row's final normaliser); a step without importance gives
+    them to the one-pass kernel, whose ordinary scores never leave its
+    exponent band."""
+    inp = workloads.generate("small_longcache")
+    n = np.diff(inp.cu_seqlens_q)
+    want = inp.n_heads * int(((n + 127) // 128).sum())
+    gpu = tl.run_gpu(inp)
+    assert gpu["layer"].last_step_work() == (want, want, 0)
+    g = tl.run_gpu(inp, want_importance=False)
+    assert g["layer"].last_step_work() == (want, 0, 0)
+
+
+@pytest.mark.parametrize("name,seqs", [("small_varlen", None), ("small_longcache", None),
+                                       ("layer_b1", None)])
+def test_one_pass_attention_without_importance(name, seqs):
+    """The one-pass kernel (steps without importance) against the oracle."""
+    inp = workloads.generate(name)
+    gpu = tl.run_gpu(inp, want_importance=False)
+    assert gpu["err"] == 0
+    ref = tl.run_oracle(inp, seqs=seqs)
+    tl.compare_step(inp, gpu, ref, seqs if seqs is not None else range(inp.batch))
+    tl.assert_unwritten_rows_unchanged(inp, gpu)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,seqs", [("batch32_uniform", [0, 13, 31]),
+                                       ("batch32_varlen", [0, 5, 17, 30]),
+                                       ("sweep_b2_m256_L8192", [0, 1])])
+def test_one_pass_attention_without_importance_full_size(name, seqs):
+    """Full-size workloads through the one-pass kernel, sampled sequences."""
+    inp = workloads.generate(name)
+    gpu = tl.run_gpu(inp, want_importance=False)
+    assert gpu["err"] == 0
+    ref = tl.run_oracle(inp, seqs=seqs)
+    tl.compare_step(inp, gpu, ref, seqs)
+    assert np.isfinite(gpu["out"]).all()
+
+
+def _plant_far_key(inp, b, n_rows, seed):
+    """Keep the first n_rows query rows of sequence b and plant, in a prior cache
+    row of its second key tile, a key whose score against every kept row is
+    +-200 (log2 units, the kernels' score domain), chosen per head as the
+    least-norm solution of q_r . k = +-200 sqrt(d) / log2(e) (rotated q of the
+    oracle).  Rows at +200 put all their attention on that key, far outside the
+    one-pass kernel's band above the first tile's maximum (2^64); rows at -200
+    ignore it.  Either way the softmax does not depend on the rounding of q,
+    which a large key magnifies (the kernels keep q in bf16)."""
+    qs = inp.seq_slice_q(b)
+    keep = np.r_[0:qs.start + n_rows, qs.stop:inp.total_q]
+    cnt = np.diff(inp.cu_seqlens_q)
+    cnt[b] = n_rows
+    inp.x, inp.q_pos = inp.x[keep], inp.q_pos[keep]
+    inp.cu_seqlens_q = np.r_[0, np.cumsum(cnt)].astype(np.int32)
+    qs, ks = inp.seq_slice_q(b), inp.seq_slice_k(b)
+    H, d = inp.n_heads, inp.head_dim
+    q, _, _ = oracle.qkv_project(inp.x[qs], inp.w_qkv, H, d)
+    q = oracle.rope_rotate(q, inp.q_pos[qs], inp.rope_theta)
+    sgn = np.random.default_rng(seed).choice([-1.0, 1.0], size=n_rows)
+    target = sgn * 200.0 * np.sqrt(d) / np.log2(np.e)
+    written = set(inp.q_pos[qs].tolist())
+    j = next(p for p in range(128, ks.stop - ks.start) if p not in written)
+    inp.k_cache = inp.k_cache.copy()
+    for h in range(H):
+        qh = q[:, h, :]
+        inp.k_cache[ks.start + j, h] = qh.T @ np.linalg.solve(qh @ qh.T, target)
+    inp.k_cache[ks.start + j] = workloads.to_bf16_exact(inp.k_cache[ks.start + j])
+    return j, sgn
+
+
+@pytest.mark.parametrize("seq", [0, 2])
+def test_scores_out_of_the_one_pass_band_are_handed_over(seq):
+    """In a step without importance, items with scores far above their first key
+    tile's maximum are handed to the two-pass kernel and still match the
+    oracle."""
+    inp = workloads.generate("small_varlen")
+    _plant_far_key(inp, seq, 64, seed=seq)
+    gpu = tl.run_gpu(inp, want_importance=False)
+    assert gpu["err"] == 0
+    items, two_pass, handed = gpu["layer"].last_step_work()
+    assert two_pass == 0 and handed == inp.n_heads  # every head of that sequence
+    ref = tl.run_oracle(inp)
+    tl.compare_step(inp, gpu, ref, range(inp.batch))
+    # with importance the same step runs in the two-pass kernel from the start
+    g2 = tl.run_gpu(inp)
+    assert g2["layer"].last_step_work()[2] == 0
+    tl.compare_step(inp, g2, ref, range(inp.batch))
 
 
 def test_topk_kernel_is_exact_on_gpu_importance():

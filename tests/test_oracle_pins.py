@@ -313,7 +313,8 @@ def test_topk_pads_when_fewer_candidates():
 
 
 # ----------------------------------------------------------------- workloads
-@pytest.mark.parametrize("name", ["tiny_fp32", "layer_b1", "small_varlen", "small_d64"])
+@pytest.mark.parametrize("name", ["tiny_fp32", "layer_b1", "small_varlen", "small_d64",
+                                  "small_longcache"])
 def test_workload_structure(name):
     inp = workloads.generate(name)
     assert inp.cu_seqlens_q[0] == 0 and inp.cu_seqlens_k[0] == 0
