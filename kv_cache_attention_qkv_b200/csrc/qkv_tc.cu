@@ -24,6 +24,8 @@
 //              stores, while the MMA warp already fills the other accumulator.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "fc_internal.h"
 #include "ptx.cuh"
 
@@ -39,13 +41,13 @@ constexpr uint32_t B_BYTES = (BN / 2) * BK * 2; // 16 KiB: this CTA's half of th
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 static_assert(kQkvXBoxRows == BM && kQkvWBoxRows == BN / 2,
               "the host's TMA boxes must match the per-CTA tiles");
-constexpr int GROUP_M = 8;                      // tile raster: groups of 8 pair row blocks
 constexpr uint32_t IDESC = ptx::idesc_bf16_f32(PM, BN, 0, 0);
 constexpr int THREADS = 192;
 
 struct QkvParams {
   int T, S, D, H;
   int num_m, num_n, num_tiles, num_k;
+  int group_m;  // tile raster: groups of this many pair row blocks
   const int32_t* q_pos;
   const int32_t* row_dst;
   const float* rcos;
@@ -64,11 +66,15 @@ struct __align__(8) Bars {
   int abort_flag;
 };
 
-__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& m, int& n) {
-  const int per_group = GROUP_M * num_n;
+// Tile t of the raster: row blocks vary fastest inside a group of group_m of
+// them, which sweeps every column block of W before the next group starts, so
+// a group's rows of X stay in L2 while W streams through once per group.
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int group_m, int& m,
+                                            int& n) {
+  const int per_group = group_m * num_n;
   const int g = t / per_group;
-  const int first_m = g * GROUP_M;
-  const int gsize = min(num_m - first_m, GROUP_M);
+  const int first_m = g * group_m;
+  const int gsize = min(num_m - first_m, group_m);
   const int r = t - g * per_group;
   m = first_m + r % gsize;
   n = r / gsize;
@@ -146,9 +152,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t phase = 0;
       int issued_phase[STAGES];
       for (int s = 0; s < STAGES; ++s) issued_phase[s] = -1;
+      // X is reused by every column block of its group, W once per group
+      const uint64_t pol_x = ptx::l2_policy_evict_last(), pol_w = ptx::l2_policy_evict_first();
       for (int t = pair; t < p.num_tiles && !failed; t += npairs) {
         int m, n;
-        tile_coords(t, p.num_m, p.num_n, m, n);
+        tile_coords(t, p.num_m, p.num_n, p.group_m, m, n);
         for (int kb = 0; kb < p.num_k; ++kb) {
           if (!ptx::mbar_wait(bar(bars->empty[stage]), phase ^ 1u, abort_flag)) {
             failed = true;
@@ -157,8 +165,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           // the leader's barrier counts both CTAs' bytes
           if (leader) ptx::mbar_arrive_expect_tx(bar(bars->full[stage]), 2 * STAGE_BYTES);
           const uint32_t lbar = ptx::mapa_shared(bar(bars->full[stage]), 0);
-          ptx::tma_load_2d_pair(sA(stage), &tm_x, kb * BK, m * PM + (int)rank * BM, lbar);
-          ptx::tma_load_2d_pair(sB(stage), &tm_w, kb * BK, n * BN + (int)rank * (BN / 2), lbar);
+          ptx::tma_load_2d_pair_hint(sA(stage), &tm_x, kb * BK, m * PM + (int)rank * BM, lbar,
+                                     pol_x);
+          ptx::tma_load_2d_pair_hint(sB(stage), &tm_w, kb * BK, n * BN + (int)rank * (BN / 2),
+                                     lbar, pol_w);
           issued_phase[stage] = (int)phase;
           if (++stage == STAGES) {
             stage = 0;
@@ -234,7 +244,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t tempty_leader1 = ptx::mapa_shared(bar(bars->tempty[1]), 0);
     for (int t = pair; t < p.num_tiles; t += npairs, ++it) {
       int m, n;
-      tile_coords(t, p.num_m, p.num_n, m, n);
+      tile_coords(t, p.num_m, p.num_n, p.group_m, m, n);
       const int a = it & 1;
       const uint32_t u = (uint32_t)(it >> 1);
       if (!ptx::mbar_wait(bar(bars->tfull[a]), u & 1u, abort_flag)) {
@@ -331,6 +341,10 @@ cudaError_t launch_qkv_tc(const fc_handle* h, cudaStream_t st, const StepShape& 
   p.num_n = 3 * s.H * HD / BN;
   p.num_tiles = p.num_m * p.num_n;
   p.num_k = s.D / BK;
+  // as many row blocks per group as keep about 48 MiB of X in L2
+  const size_t x_block_bytes = (size_t)PM * s.D * 2;
+  p.group_m = (int)std::max<size_t>(1, std::min<size_t>((size_t)p.num_m,
+                                                        (48ull << 20) / x_block_bytes));
   p.q_pos = q_pos;
   p.row_dst = h->ws.row_dst;
   p.rcos = h->ws.rope_cos;
