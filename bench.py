@@ -239,8 +239,32 @@ def _dist_env():
     return ws, rank, local
 
 
+def _work_balance(inp, num_ctas, qtile=128, ktile=128):
+    """Balance of the attention kernels' static schedule: the work list holds
+    one item per (sequence, head, 128-row query tile), longest caches first;
+    in round r CTA c takes item r * num_ctas + c (even r) or
+    r * num_ctas + num_ctas - 1 - c (odd r); an item's cost is taken as its
+    number of 128-key tiles."""
+    n = np.diff(inp.cu_seqlens_q).astype(np.int64)
+    L = np.diff(inp.cu_seqlens_k).astype(np.int64)
+    order = sorted(range(inp.batch), key=lambda b: (-int(L[b]), b))
+    cost = []
+    for b in order:
+        if n[b] > 0 and L[b] > 0:
+            cost += [int((L[b] + ktile - 1) // ktile)] * (inp.n_heads * int((n[b] + qtile - 1) // qtile))
+    per = np.zeros(num_ctas, np.int64)
+    for i, c in enumerate(cost):
+        r, k = divmod(i, num_ctas)
+        per[num_ctas - 1 - k if r % 2 else k] += c
+    return {"items": len(cost), "ctas": num_ctas, "tiles_max_per_cta": int(per.max()),
+            "tiles_mean_per_cta": float(per.mean()),
+            "max_over_mean": float(per.max() / per.mean()) if per.mean() else None,
+            "note": "static alternating-direction schedule over the longest-first work "
+                    "list; cost = key tiles per item"}
+
+
 def _step_result(args, inp, ws, *, total_ms, burst_ms, per_kernel, launches, err, e2e_ms, h2d,
-                 d2h, clocks):
+                 d2h, clocks, noimp=None, num_sms=148):
     """The JSON line of a step run from its measurements (no GPU needed).
 
     per_kernel: {name: (total ms, launches)} of the per-kernel pass; total_ms,
@@ -248,9 +272,13 @@ def _step_result(args, inp, ws, *, total_ms, burst_ms, per_kernel, launches, err
     peaks = _peaks()
     wk = _work(inp)
     T = inp.total_q
-    # a step with importance runs the two-pass attention kernel alone; the
-    # one-pass kernel (steps without importance) is timed in its own slot
+    # a step with importance runs the two-pass attention kernel alone; a step
+    # without runs the one-pass kernel and the two-pass kernel for the items it
+    # hands over (usually none): its attention is the sum of the two
     per_kernel = dict(per_kernel)
+    if getattr(args, "no_importance", False) and "attention_one_pass" in per_kernel:
+        (ma, na), (mb, _) = per_kernel["attention_one_pass"], per_kernel["attention"]
+        per_kernel["attention"] = (ma + mb, na)
     ms_per_step = total_ms / args.steps
     tokens = T * ws * args.steps
     value = tokens / (total_ms / 1e3)
@@ -260,11 +288,22 @@ def _step_result(args, inp, ws, *, total_ms, burst_ms, per_kernel, launches, err
     traffic = _dram_traffic(args.workload)
     sm_mhz = (clocks or {}).get("sm_mhz")
     rl = _kernel_roofline(dom, *names[dom], per_kernel[dom], peaks, traffic.get(dom), sm_mhz)
+    extra = {}
+    if noimp is not None:
+        nms, npk = noimp
+        one = npk.get("attention_one_pass", (0.0, 0))
+        extra["no_importance"] = {
+            "ms_per_step": nms / args.steps, "value": T * ws * args.steps / (nms / 1e3),
+            "kernels_ms_per_step": {k: v[0] / max(v[1], 1) for k, v in npk.items() if v[1]},
+            "attention_one_pass": (_kernel_roofline("attention_one_pass", "hbm", wk["attn_bytes"],
+                                                    one, peaks, None, sm_mhz) if one[1] else None),
+            "note": "context: the same step without importance or reselection; its attention "
+                    "runs in the one-pass kernel"}
     return {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": inp.dtype, "data": "synthetic",
-        "config": _step_config(args.workload, inp, ws),
+        "config": _step_config(args.workload, inp, ws, not getattr(args, "no_importance", False)),
         "roofline": {"kernel": dom, "bound": rl["bound"], "achieved": rl["achieved"],
                      "peak": rl["peak"], "unit": rl["unit"], "frac": rl["frac"],
                      "traffic": rl["traffic"], "frac_vs": rl["frac_vs"],
@@ -282,6 +321,8 @@ def _step_result(args, inp, ws, *, total_ms, burst_ms, per_kernel, launches, err
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "clocks": clocks,
+        "work_balance": _work_balance(inp, num_sms),
+        **extra,
     }
 
 
@@ -325,10 +366,16 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     def step():
+        if args.no_importance:  # attention only (the one-pass kernel), no reselection
+            layer.step(x, qp, cq, ck, kc, vc, out, None)
+            return layer.last_launch_count
         layer.step(x, qp, cq, ck, kc, vc, out, imp)
         n = layer.last_launch_count
         layer.topk_tracked(imp, ck, lo, hi, K, tracked, k_per_seq=kps)
         return n + layer.last_launch_count
+
+    def step_noimp():
+        layer.step(x, qp, cq, ck, kc, vc, out, None)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -388,6 +435,28 @@ def run_ours(args):
             step()
         torch.cuda.synchronize()
         per_kernel = layer.profile_read()
+        # context: the same step without importance (its attention runs in the
+        # one-pass kernel), step time and per-kernel times
+        noimp = None
+        if not args.no_importance:
+            layer.profile(False)
+            torch.cuda.synchronize()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            for k in range(args.steps):
+                flush.fill_(float(k))
+                ev[k][0].record(stream)
+                step_noimp()
+                ev[k][1].record(stream)
+            torch.cuda.synchronize()
+            noimp_ms = sum(a.elapsed_time(b) for a, b in ev)
+            layer.profile(True)
+            layer.profile_read()
+            for k in range(args.steps):
+                flush.fill_(float(k))
+                step_noimp()
+            torch.cuda.synchronize()
+            noimp = (noimp_ms, layer.profile_read())
         layer.profile(False)
         clk.window_end()
     total_ms = float(sum(step_ms))
@@ -432,7 +501,8 @@ def run_ours(args):
     if rank == 0:
         result = _step_result(args, inp, ws, total_ms=total_ms, burst_ms=burst_ms,
                               per_kernel=per_kernel, launches=launches, err=err, e2e_ms=e2e_ms,
-                              h2d=h2d, d2h=d2h, clocks=clk.summary())
+                              h2d=h2d, d2h=d2h, clocks=clk.summary(), noimp=noimp,
+                              num_sms=torch.cuda.get_device_properties(dev).multi_processor_count)
         # the oracle's timing is a single-GPU line's context: rank 0 at N = 1 only
         result["cpu_baseline"] = (cpu_baseline(inp, budget_s=args.cpu_budget)
                                   if args.cpu_budget > 0 and ws == 1 else None)
@@ -453,9 +523,10 @@ def _oracle_threads():
         return os.cpu_count()
 
 
-def _step_config(workload, inp, ws):
+def _step_config(workload, inp, ws, importance=True):
     """The workload description both arms print (the same keys at every N)."""
-    return {"workload": workload, "batch": inp.batch, "seq_len": int(np.diff(inp.cu_seqlens_k).max()),
+    extra = {} if importance else {"importance": False}
+    return {**extra, "workload": workload, "batch": inp.batch, "seq_len": int(np.diff(inp.cu_seqlens_k).max()),
             "query_rows_per_seq": int(np.diff(inp.cu_seqlens_q).max()), "hidden": inp.hidden,
             "heads": inp.n_heads, "head_dim": inp.head_dim, "topk": int(inp.topk.max()),
             "total_q": inp.total_q, "total_k": inp.total_k,
@@ -713,6 +784,9 @@ def main():
                     help="time draft-and-verify decode iterations of the model (one JSON line)")
     ap.add_argument("--model", action="store_true",
                     help="time the 32-layer model step around the layer (one JSON line)")
+    ap.add_argument("--no-importance", action="store_true",
+                    help="time fc_step without importance or reselection (the one-pass attention "
+                         "kernel); for profiling, not the headline")
     ap.add_argument("--sweep", choices=sorted(SWEEPS) + ["all"], default=None,
                     help="time every point of a sweep axis (one JSON line per point, no cpu_baseline)")
     args = ap.parse_args()

@@ -218,10 +218,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         return true;
       };
       // the next item's record is fetched while this one runs
-      WorkItem wnext = fetch_item(p, first, n_items, blockIdx.x);
-      for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
+      WorkItem wnext = fetch_item(p, first, n_items, snake_item(0, blockIdx.x, gridDim.x));
+      for (int r = 0, it = snake_item(0, blockIdx.x, gridDim.x); it < n_items && !failed;
+         ++r, it = snake_item(r, blockIdx.x, gridDim.x), ++ic) {
         const Item t = to_item(wnext);
-        wnext = fetch_item(p, first, n_items, it + gridDim.x);
+        wnext = fetch_item(p, first, n_items, snake_item(r + 1, blockIdx.x, gridDim.x));
         if (!ptx::mbar_wait(bar(bars->qfree), (ic & 1u) ^ 1u, abort_flag)) {
           failed = true;
           break;
@@ -305,10 +306,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         return true;
       };
       // the next item's record is fetched while this one runs
-      WorkItem wnext = fetch_item(p, first, n_items, blockIdx.x);
-      for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
+      WorkItem wnext = fetch_item(p, first, n_items, snake_item(0, blockIdx.x, gridDim.x));
+      for (int r = 0, it = snake_item(0, blockIdx.x, gridDim.x); it < n_items && !failed;
+         ++r, it = snake_item(r, blockIdx.x, gridDim.x), ++ic) {
         const Item t = to_item(wnext);
-        wnext = fetch_item(p, first, n_items, it + gridDim.x);
+        wnext = fetch_item(p, first, n_items, snake_item(r + 1, blockIdx.x, gridDim.x));
         if (!ptx::mbar_wait(bar(bars->qfull), ic & 1u, abort_flag)) {
           failed = true;
           break;
@@ -366,8 +368,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                  ? __ldg(reinterpret_cast<const int*>(p.items + first + idx) + lane)
                  : 0;
     };
-    int fnext = fetch_field(blockIdx.x);
-    for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
+    int fnext = fetch_field(snake_item(0, blockIdx.x, gridDim.x));
+    for (int r = 0, it = snake_item(0, blockIdx.x, gridDim.x); it < n_items && !failed;
+         ++r, it = snake_item(r, blockIdx.x, gridDim.x), ++ic) {
       WorkItem wcur;
       wcur.seq = __shfl_sync(0xffffffffu, fnext, 0);
       wcur.tile_head = __shfl_sync(0xffffffffu, fnext, 1);
@@ -376,7 +379,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       wcur.k0 = __shfl_sync(0xffffffffu, fnext, 4);
       wcur.L = __shfl_sync(0xffffffffu, fnext, 5);
       const Item t = to_item(wcur);
-      fnext = fetch_field(it + gridDim.x);
+      fnext = fetch_field(snake_item(r + 1, blockIdx.x, gridDim.x));
       const int par = (int)(ic & 1u);
       const bool row_ok = rl < t.nrows;
       float M = 0.f, l = 0.f, smax = -INFINITY;

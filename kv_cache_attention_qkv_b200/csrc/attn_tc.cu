@@ -241,10 +241,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         return true;
       };
       // the next item's record is fetched while this one runs
-      WorkItem wnext = fetch_item(p, n_long, n_items, blockIdx.x);
-      for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
+      WorkItem wnext = fetch_item(p, n_long, n_items, snake_item(0, blockIdx.x, gridDim.x));
+      for (int r = 0, it = snake_item(0, blockIdx.x, gridDim.x); it < n_items && !failed;
+         ++r, it = snake_item(r, blockIdx.x, gridDim.x), ++ic) {
         const Item t = to_item(wnext);
-        wnext = fetch_item(p, n_long, n_items, it + gridDim.x);
+        wnext = fetch_item(p, n_long, n_items, snake_item(r + 1, blockIdx.x, gridDim.x));
         if (!ptx::mbar_wait(bar(bars->qfree), (ic & 1u) ^ 1u, abort_flag)) {
           failed = true;
           break;
@@ -326,10 +327,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         return true;
       };
       // the next item's record is fetched while this one runs
-      WorkItem wnext = fetch_item(p, n_long, n_items, blockIdx.x);
-      for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
+      WorkItem wnext = fetch_item(p, n_long, n_items, snake_item(0, blockIdx.x, gridDim.x));
+      for (int r = 0, it = snake_item(0, blockIdx.x, gridDim.x); it < n_items && !failed;
+         ++r, it = snake_item(r, blockIdx.x, gridDim.x), ++ic) {
         const Item t = to_item(wnext);
-        wnext = fetch_item(p, n_long, n_items, it + gridDim.x);
+        wnext = fetch_item(p, n_long, n_items, snake_item(r + 1, blockIdx.x, gridDim.x));
         if (!ptx::mbar_wait(bar(bars->qfull), ic & 1u, abort_flag)) {
           failed = true;
           break;
@@ -436,8 +438,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                  ? __ldg(reinterpret_cast<const int*>(item_ptr(p, n_long, it)) + lane)
                  : 0;
     };
-    int fnext = fetch_field(blockIdx.x);
-    for (int it = blockIdx.x; it < n_items && !failed; it += gridDim.x, ++ic) {
+    int fnext = fetch_field(snake_item(0, blockIdx.x, gridDim.x));
+    for (int r = 0, it = snake_item(0, blockIdx.x, gridDim.x); it < n_items && !failed;
+         ++r, it = snake_item(r, blockIdx.x, gridDim.x), ++ic) {
       WorkItem wcur;
       wcur.seq = __shfl_sync(0xffffffffu, fnext, 0);
       wcur.tile_head = __shfl_sync(0xffffffffu, fnext, 1);
@@ -446,7 +449,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       wcur.k0 = __shfl_sync(0xffffffffu, fnext, 4);
       wcur.L = __shfl_sync(0xffffffffu, fnext, 5);
       const Item t = to_item(wcur);
-      fnext = fetch_field(it + gridDim.x);
+      fnext = fetch_field(snake_item(r + 1, blockIdx.x, gridDim.x));
       uint32_t sv[64];
       // ---- pass 1: max and normaliser over this warp's tiles and column half
       float m = -INFINITY, l = 0.f;

@@ -31,6 +31,7 @@ struct GemmParams {
   int mode;
   int M, N, K;     // rows of A, output columns (SwiGLU: features), reduction length
   int num_m, num_n, num_tiles, num_k;  // filled by the launcher
+  int group_m;                         // tile raster (launcher): row blocks per group
   const __nv_bfloat16* resid;  // GEMM_RESID: [M, ldo] added to the product (may equal out)
   __nv_bfloat16* out;          // GEMM_RESID / GEMM_SWIGLU: [M, ldo]
   size_t ldo;                  // row stride of resid / out in elements
@@ -56,6 +57,14 @@ struct __align__(16) WorkItem {
   int32_t L;          // cache rows of the sequence
   int32_t pad[2];
 };
+
+// Item index of CTA `cta` in round `round` of a persistent schedule over a
+// work list ordered by decreasing cost: the rounds alternate direction (CTA c
+// takes position c, then position ctas - 1 - c), which spreads the costly
+// items more evenly than plain round-robin.
+__device__ __forceinline__ int snake_item(int round, int cta, int ctas) {
+  return round * ctas + ((round & 1) ? ctas - 1 - cta : cta);
+}
 
 struct Workspace {
   void* q_buf = nullptr;                  // [max_total_q, H, d] dtype; rotated, pre-scaled q

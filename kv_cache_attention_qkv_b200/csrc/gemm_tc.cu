@@ -22,6 +22,8 @@
 //   warps 2-5  epilogue (both CTAs): tcgen05.ld of its 32-row quadrant.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "fc_internal.h"
 #include "ptx.cuh"
 
@@ -34,7 +36,6 @@ constexpr int BN = 256, BK = 64, STAGES = 6;
 constexpr uint32_t A_BYTES = BM * BK * 2;        // 16 KiB
 constexpr uint32_t B_BYTES = (BN / 2) * BK * 2;  // 16 KiB: this CTA's half of the B tile
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int GROUP_M = 8;
 constexpr uint32_t IDESC = ptx::idesc_bf16_f32(PM, BN, 0, 0);
 constexpr int THREADS = 192;
 static_assert(kGemmBoxRows == BM && kGemmBoxRows == BN / 2, "TMA boxes must match the tiles");
@@ -45,11 +46,15 @@ struct __align__(8) Bars {
   int abort_flag;
 };
 
-__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& m, int& n) {
-  const int per_group = GROUP_M * num_n;
+// Tile t of the raster: row blocks vary fastest inside a group of group_m of
+// them, which sweeps every column block of B before the next group starts, so
+// a group's rows of A stay in L2 while B streams through once per group.
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int group_m, int& m,
+                                            int& n) {
+  const int per_group = group_m * num_n;
   const int g = t / per_group;
-  const int first_m = g * GROUP_M;
-  const int gsize = min(num_m - first_m, GROUP_M);
+  const int first_m = g * group_m;
+  const int gsize = min(num_m - first_m, group_m);
   const int r = t - g * per_group;
   m = first_m + r % gsize;
   n = r / gsize;
@@ -120,7 +125,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const CUtensorMap* tm_b = (p.mode == GEMM_SWIGLU && rank == 1) ? &tm_b1 : &tm_b0;
       for (int t = pair; t < p.num_tiles && !failed; t += npairs) {
         int m, n;
-        tile_coords(t, p.num_m, p.num_n, m, n);
+        tile_coords(t, p.num_m, p.num_n, p.group_m, m, n);
         // B rows of this CTA: its half of a 256-row tile, or for SwiGLU the
         // tile's 128 features of its own matrix (gate on the leader, up on the other)
         const int brow = p.mode == GEMM_SWIGLU ? n * (BN / 2) : n * BN + (int)rank * (BN / 2);
@@ -204,7 +209,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t tempty_leader1 = ptx::mapa_shared(bar(bars->tempty[1]), 0);
     for (int t = pair; t < p.num_tiles; t += npairs, ++it) {
       int m, n;
-      tile_coords(t, p.num_m, p.num_n, m, n);
+      tile_coords(t, p.num_m, p.num_n, p.group_m, m, n);
       const int a = it & 1;
       const uint32_t u = (uint32_t)(it >> 1);
       if (!ptx::mbar_wait(bar(bars->tfull[a]), u & 1u, abort_flag)) {
@@ -329,6 +334,10 @@ cudaError_t launch_gemm_tc(int num_sms, cudaStream_t st, const CUtensorMap& tm_a
   p.num_n = p.mode == GEMM_SWIGLU ? p.N / (BN / 2) : (p.N + BN - 1) / BN;
   p.num_tiles = p.num_m * p.num_n;
   p.num_k = p.K / BK;
+  // as many row blocks per group as keep about 48 MiB of A in L2
+  const size_t a_block_bytes = (size_t)PM * p.K * 2;
+  p.group_m = (int)std::max<size_t>(1, std::min<size_t>((size_t)p.num_m,
+                                                        (48ull << 20) / a_block_bytes));
   if (p.num_tiles == 0) return cudaSuccess;
   const size_t smem = gemm_tc_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

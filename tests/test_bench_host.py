@@ -142,3 +142,14 @@ def test_step_result_line_follows_the_contract():
     assert st["judged_on"] == "sustained_clock_scaled"
     assert rl["frac_vs"]["sustained_clock_scaled"] == pytest.approx(rl["achieved"] / scaled)
     assert rl["frac_vs"]["spec"] == pytest.approx(rl["achieved"] / bench.SPEC_BF16_TFLOPS)
+    wb = r["work_balance"]
+    assert wb["items"] == 2 and wb["tiles_max_per_cta"] == 1  # 2 heads x 1 query tile, 64 keys
+    # the no-importance context line, from made-up per-kernel times
+    noimp = (3.0, {"prep": (0.1, 10), "qkv_rope_scatter": (2.5, 10), "attention": (0.01, 10),
+                   "attention_one_pass": (0.4, 10)})
+    r2 = bench._step_result(args, inp, 2, total_ms=5.0, burst_ms=4.0, per_kernel=per_kernel,
+                            launches=50, err=0, e2e_ms=8.0, h2d=1000, d2h=2000, clocks=clocks,
+                            noimp=noimp, num_sms=148)
+    ni = r2["no_importance"]
+    assert ni["ms_per_step"] == pytest.approx(0.3)
+    assert ni["attention_one_pass"]["achieved"] == pytest.approx(wk["attn_bytes"] / 0.04e-3 / 1e9)
