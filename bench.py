@@ -264,7 +264,7 @@ def _work_balance(inp, num_ctas, qtile=128, ktile=128):
 
 
 def _step_result(args, inp, ws, *, total_ms, burst_ms, per_kernel, launches, err, e2e_ms, h2d,
-                 d2h, clocks, noimp=None, num_sms=148):
+                 d2h, clocks, noimp=None, num_sms=148, e2e_host_ms=None):
     """The JSON line of a step run from its measurements (no GPU needed).
 
     per_kernel: {name: (total ms, launches)} of the per-kernel pass; total_ms,
@@ -319,7 +319,10 @@ def _step_result(args, inp, ws, *, total_ms, burst_ms, per_kernel, launches, err
                   "note": "the same K steps right after the warm-up, before the power "
                           "controller reacts; value and rooflines above are the steady state"},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                **({"ms_per_step": e2e_ms / args.steps,
+                    "host_enqueue_ms_per_step": e2e_host_ms / args.steps}
+                   if e2e_host_ms is not None else {})},
         "clocks": clocks,
         "work_balance": _work_balance(inp, num_sms),
         **extra,
@@ -359,6 +362,7 @@ def run_ours(args):
                        max_batch=B, max_total_q=T, max_total_k=S,
                        max_seqlen_q=int(np.diff(inp.cu_seqlens_q).max()),
                        max_pos=int(np.diff(inp.cu_seqlens_k).max()), max_topk=K)
+    layer.set_qkv_kernel(args.qkv_kernel, args.qkv_split)
     out = torch.empty((T, H, d), device=dev, dtype=dt)
     imp = torch.empty((S,), device=dev, dtype=torch.float32)
     tracked = torch.empty((B, K), device=dev, dtype=torch.int32)
@@ -488,8 +492,10 @@ def run_ours(args):
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    t_host = time.perf_counter()
     for _ in range(args.steps):
         e2e_step()
+    t_host = time.perf_counter() - t_host  # host time to enqueue the K steps
     layer.host_sync()  # the stream waits for the last output copies
     e1.record(stream)
     torch.cuda.synchronize()
@@ -500,9 +506,11 @@ def run_ours(args):
     result = None
     if rank == 0:
         result = _step_result(args, inp, ws, total_ms=total_ms, burst_ms=burst_ms,
+                              e2e_host_ms=t_host * 1e3,
                               per_kernel=per_kernel, launches=launches, err=err, e2e_ms=e2e_ms,
                               h2d=h2d, d2h=d2h, clocks=clk.summary(), noimp=noimp,
                               num_sms=torch.cuda.get_device_properties(dev).multi_processor_count)
+        result["qkv_plan"] = layer.qkv_plan(T)
         # the oracle's timing is a single-GPU line's context: rank 0 at N = 1 only
         result["cpu_baseline"] = (cpu_baseline(inp, budget_s=args.cpu_budget)
                                   if args.cpu_budget > 0 and ws == 1 else None)
@@ -761,6 +769,143 @@ def run_decode(args):
     }
 
 
+def _copy_rates(torch, nbytes, dev, reps=10):
+    """GB/s of pinned host<->device copies of nbytes: each direction alone on
+    its own stream, then both at once on two streams (CUDA events)."""
+    h_in = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    h_out = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d_in = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    d_out = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    res = {}
+    for name, legs in (("h2d", [(s1, d_in, h_in)]), ("d2h", [(s2, h_out, d_out)]),
+                       ("both", [(s1, d_in, h_in), (s2, h_out, d_out)])):
+        for _ in range(2):
+            for st, dst, src in legs:
+                with torch.cuda.stream(st):
+                    dst.copy_(src, non_blocking=True)
+        torch.cuda.synchronize()
+        evs = []
+        for st, dst, src in legs:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            with torch.cuda.stream(st):
+                for _ in range(reps):
+                    dst.copy_(src, non_blocking=True)
+            b.record(st)
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        res[name] = [nbytes * reps / (a.elapsed_time(b) / 1e3) / 1e9 for a, b in evs]
+    return {"h2d_gbs": res["h2d"][0], "d2h_gbs": res["d2h"][0],
+            "both_h2d_gbs": res["both"][0], "both_d2h_gbs": res["both"][1], "bytes": nbytes}
+
+
+def run_e2e_timeline(args):
+    """Per-stage timeline of the end-to-end step (fc_step_host): the input
+    copies and output copies on the handle's copy streams and the kernels on
+    the compute stream, recorded with CUDA events for K steps after W warm-up
+    steps, plus the bare copy rates of the same sizes."""
+    import torch
+
+    from kv_cache_attention_qkv_b200 import FlashCache, workloads
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    inp = workloads.generate(args.workload)
+    dt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
+    f = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dtype=dt)
+    w, kc, vc = f(inp.w_qkv), f(inp.k_cache), f(inp.v_cache)
+    T, S, H, d, B = inp.total_q, inp.total_k, inp.n_heads, inp.head_dim, inp.batch
+    K = int(inp.topk.max())
+    layer = FlashCache(w, hidden=inp.hidden, n_heads=H, head_dim=d, rope_theta=inp.rope_theta,
+                       max_batch=B, max_total_q=T, max_total_k=S,
+                       max_seqlen_q=int(np.diff(inp.cu_seqlens_q).max()),
+                       max_pos=int(np.diff(inp.cu_seqlens_k).max()), max_topk=K)
+    x_h = torch.from_numpy(np.ascontiguousarray(inp.x)).to(dt).pin_memory()
+    small_h = {n: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).pin_memory()
+               for n, a in (("q_pos", inp.q_pos), ("cu_q", inp.cu_seqlens_q), ("cu_k", inp.cu_seqlens_k),
+                            ("lo", inp.cand_lo), ("hi", inp.cand_hi), ("kps", inp.topk))}
+    out_h = torch.empty((T, H, d), dtype=dt).pin_memory()
+    tr_h = torch.empty((B, K), dtype=torch.int32).pin_memory()
+
+    def e2e_step():
+        layer.step_host(x_h, small_h["q_pos"], small_h["cu_q"], small_h["cu_k"], kc, vc,
+                        small_h["lo"], small_h["hi"], K, out_h, tr_h, k_per_seq=small_h["kps"])
+
+    for _ in range(args.warmup):
+        e2e_step()
+    layer.host_sync()
+    torch.cuda.synchronize()
+    if args.soak > 0:  # the steady state of a sustained load, as the main bench times it
+        t0, n_ = time.perf_counter(), 0
+        while time.perf_counter() - t0 < args.soak:
+            e2e_step()
+            n_ += 1
+            if n_ % 16 == 0:
+                layer.host_sync()
+                torch.cuda.synchronize()
+        layer.host_sync()
+        torch.cuda.synchronize()
+    # the same K steps timed as the main bench times them (no per-stage events)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    layer.host_sync()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    plain_ms = e0.elapsed_time(e1) / args.steps
+    layer.profile(True)
+    layer.profile_read()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    layer.host_sync()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    profiled_ms = e0.elapsed_time(e1) / args.steps
+    tl_ = layer.profile_timeline()
+    layer.profile_read()
+    layer.profile(False)
+    layer.close()
+    # group the records by step: every step has one h2d_copy record
+    steps, cur = [], None
+    for name, a, b in tl_:
+        if name == "h2d_copy":
+            cur = {"h2d": (a, b), "kernels": [], "d2h": None}
+            steps.append(cur)
+        elif name == "d2h_copy":
+            cur["d2h"] = (a, b)
+        else:
+            cur["kernels"].append((a, b))
+    mid = steps[2:-2] if len(steps) > 6 else steps
+    mean = lambda xs: float(np.mean(xs)) if xs else None
+    h2d = [s_["h2d"][1] - s_["h2d"][0] for s_ in mid]
+    d2h = [s_["d2h"][1] - s_["d2h"][0] for s_ in mid]
+    comp = [s_["kernels"][-1][1] - s_["kernels"][0][0] for s_ in mid]
+    period = [b_["h2d"][0] - a_["h2d"][0] for a_, b_ in zip(mid, mid[1:])]
+    # time each copy of step n overlaps the other direction's copies
+    def overlap(a, others):
+        return sum(max(0.0, min(a[1], o[1]) - max(a[0], o[0])) for o in others)
+    ov = [overlap(s_["h2d"], [t_["d2h"] for t_ in steps]) / (s_["h2d"][1] - s_["h2d"][0]) for s_ in mid]
+    h2d_bytes = x_h.numel() * x_h.element_size() + sum(t.numel() * 4 for t in small_h.values())
+    d2h_bytes = out_h.numel() * out_h.element_size() + tr_h.numel() * 4
+    rates = _copy_rates(torch, int(x_h.numel() * x_h.element_size()), dev)
+    return {
+        "metric": "end-to-end step timeline (fc_step_host)", "workload": args.workload,
+        "steps": args.steps, "warmup": args.warmup, "soak_s": args.soak, "steps_analysed": len(mid),
+        "ms_per_step_without_events": plain_ms, "ms_per_step_with_events": profiled_ms,
+        "period_ms": mean(period), "h2d_copy_ms": mean(h2d), "d2h_copy_ms": mean(d2h),
+        "kernels_ms": mean(comp), "h2d_bytes": int(h2d_bytes), "d2h_bytes": int(d2h_bytes),
+        "h2d_gbs_in_step": h2d_bytes / (mean(h2d) / 1e3) / 1e9,
+        "d2h_gbs_in_step": d2h_bytes / (mean(d2h) / 1e3) / 1e9,
+        "h2d_overlapped_by_d2h": mean(ov), "bare_copy_rates": rates,
+        "note": "per-kernel events on the compute stream stop the programmatic overlap of its "
+                "kernels, so kernels_ms is a little above the step's device time",
+    }
+
+
 # Sweep axes (the pages' measured axes, throughput side): batch size at the
 # headline query and cache, query size beta_m at batch 32, cache length at
 # batch 32 and beta_m 128.
@@ -784,9 +929,17 @@ def main():
                     help="time draft-and-verify decode iterations of the model (one JSON line)")
     ap.add_argument("--model", action="store_true",
                     help="time the 32-layer model step around the layer (one JSON line)")
+    ap.add_argument("--e2e-timeline", action="store_true",
+                    help="per-stage timeline of the end-to-end (host-buffer) step (one JSON line)")
+    ap.add_argument("--soak", type=float, default=0.0,
+                    help="with --e2e-timeline: seconds of the same end-to-end steps first")
     ap.add_argument("--no-importance", action="store_true",
                     help="time fc_step without importance or reselection (the one-pass attention "
                          "kernel); for profiling, not the headline")
+    ap.add_argument("--qkv-kernel", choices=["auto", "pair", "splitk"], default="auto",
+                    help="projection kernel of the tensor-core path (default: the CTA-pair kernel)")
+    ap.add_argument("--qkv-split", type=int, default=0,
+                    help="cluster size of the split-K projection (default: the largest that fits at once)")
     ap.add_argument("--sweep", choices=sorted(SWEEPS) + ["all"], default=None,
                     help="time every point of a sweep axis (one JSON line per point, no cpu_baseline)")
     args = ap.parse_args()
@@ -794,6 +947,9 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.model:
         print(json.dumps(run_model(args)), flush=True)
+        return
+    if args.e2e_timeline:
+        print(json.dumps(run_e2e_timeline(args)), flush=True)
         return
     if args.decode:
         print(json.dumps(run_decode(args)), flush=True)

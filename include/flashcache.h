@@ -255,24 +255,71 @@ FC_API fc_status fc_last_step_work(fc_handle* h, int32_t* items, int32_t* two_pa
  */
 FC_API const char* fc_last_cuda_error(const fc_handle* h);
 
+/*
+ * fc_set_option — select among equivalent implementations (results agree
+ * within the parity bar; for tests and measurement).
+ *   FC_OPT_QKV_KERNEL: the projection kernel of the bf16 tensor-core path:
+ *     0 (default) and 1: the CTA-pair kernel (256-row tiles, the whole
+ *       reduction per pair); 2: the split-K kernel (128-row tiles, the
+ *       reduction split over a thread-block cluster).  The split-K kernel
+ *       was measured no faster than the pair kernel on any shape tried, so
+ *       the default does not choose it.
+ *   FC_OPT_QKV_SPLIT: CTAs per cluster of the split-K kernel, 1..8, or 0
+ *     (default) to choose by occupancy.  The reduction over the hidden size is
+ *     cut into that many nearly equal runs of 64-wide steps; a value above
+ *     hidden / 64 leaves some CTAs without a step and is rejected at fc_step
+ *     with FC_ERR_INVALID_ARG.
+ * FC_ERR_INVALID_ARG for an unknown option or value.
+ */
+#define FC_OPT_QKV_KERNEL 1
+#define FC_OPT_QKV_SPLIT 2
+FC_API fc_status fc_set_option(fc_handle* h, int option, int value);
+
+/*
+ * fc_qkv_plan — the projection kernel fc_step launches for total_q query rows
+ * under the current options (host only, no GPU work).
+ *   *kernel: 0 the CUDA-core path (shapes outside the tensor-core kernels),
+ *            1 the CTA-pair kernel (256-row tiles, whole reduction per pair),
+ *            2 the split-K kernel (128-row tiles, the reduction split over a
+ *              thread-block cluster of *split CTAs, partial sums added through
+ *              distributed shared memory).
+ *   *split: CTAs per cluster for kernel 2, else 0.
+ *   *max_clusters (may be NULL): clusters of that size the GPU holds at once
+ *     (when the plan is not kernel 2: of the largest split it considered);
+ *     a negative value is the CUDA error code of the occupancy query, negated.
+ * With kernel 2 forced and no split forced, the split is the largest (at most
+ * 8 and hidden / 64) whose clusters all fit on the GPU at once.
+ * FC_ERR_INVALID_ARG for a null handle or output, total_q < 0.
+ */
+FC_API fc_status fc_qkv_plan(const fc_handle* h, int total_q, int* kernel, int* split,
+                             int* max_clusters);
+
 /* Number of kernels the last fc_step / fc_topk_tracked call enqueued (host). */
 FC_API int fc_last_launch_count(const fc_handle* h);
 
 /*
  * Per-kernel timing for measurement tools.  fc_profile(h, 1) makes every later
- * fc_step / fc_topk_tracked record a CUDA event pair on its stream around each
- * kernel it launches (up to 4096 launches); fc_profile(h, 0) stops recording.
- * fc_profile_read waits for the recorded work, writes for each kernel slot
+ * fc_step / fc_topk_tracked / fc_step_host record a CUDA event pair on its
+ * stream around each kernel it launches, and fc_step_host also around its
+ * input copies and its output copies on its copy streams (up to 4096 records);
+ * fc_profile(h, 0) stops recording.
+ * fc_profile_read waits for the recorded work, writes for each slot
  * (0 prep, 1 qkv_rope_scatter, 2 attention (the two-pass attention kernel
  * of the tensor-core path: every item of a step with importance, the items
  * handed over in a step without), 3 importance_finalize, 4 topk,
  * 5 attention_one_pass (the one-pass kernel of a tensor-core step without
- * importance)) the summed milliseconds to ms[slot] and the launch count to
- * launches[slot] (host arrays of FC_PROFILE_SLOTS entries), and clears the
- * record.
+ * importance), 6 h2d_copy and 7 d2h_copy (the copy blocks of fc_step_host))
+ * the summed milliseconds to ms[slot] and the record count to launches[slot]
+ * (host arrays of FC_PROFILE_SLOTS entries), and clears the records.
+ * fc_profile_timeline (call it before fc_profile_read) waits for the recorded
+ * work and writes, for the first min(max_records, count) records in recording
+ * order, the slot and the start and end times in milliseconds after the first
+ * record's start (host arrays); *n receives the number written.
  */
-#define FC_PROFILE_SLOTS 6
+#define FC_PROFILE_SLOTS 8
 FC_API fc_status fc_profile(fc_handle* h, int enable);
+FC_API fc_status fc_profile_timeline(fc_handle* h, int max_records, int32_t* slot, float* start_ms,
+                                     float* end_ms, int* n);
 FC_API fc_status fc_profile_read(fc_handle* h, float* ms, int* launches);
 
 /*

@@ -27,9 +27,9 @@ EXPORTED = ("fc_create", "fc_step", "fc_topk_tracked", "fc_step_host", "fc_host_
             "fc_attention_noalloc", "fc_selftest_wait_timeout", "fc_destroy", "fc_status_str",
             "fc_model_create", "fc_model_step", "fc_model_layer_handle", "fc_model_destroy",
             "fc_decode_iteration", "fc_model_lm_head", "fc_last_step_work",
-            "fc_last_cuda_error")
+            "fc_last_cuda_error", "fc_profile_timeline", "fc_set_option", "fc_qkv_plan")
 PROFILE_SLOTS = ("prep", "qkv_rope_scatter", "attention", "importance_finalize", "topk",
-                 "attention_one_pass")
+                 "attention_one_pass", "h2d_copy", "d2h_copy")
 
 
 class FlashCacheError(RuntimeError):
@@ -83,6 +83,10 @@ def load_library(path: Optional[str] = None):
     lib.fc_step_host.restype = c_int
     lib.fc_host_sync.argtypes = [vp, vp]
     lib.fc_host_sync.restype = c_int
+    lib.fc_qkv_plan.argtypes = [vp, c_int, i32p, i32p, i32p]
+    lib.fc_qkv_plan.restype = c_int
+    lib.fc_set_option.argtypes = [vp, c_int, c_int]
+    lib.fc_set_option.restype = c_int
     lib.fc_last_cuda_error.argtypes = [vp]
     lib.fc_last_cuda_error.restype = ctypes.c_char_p
     lib.fc_last_step_work.argtypes = [vp, i32p, i32p, i32p]
@@ -94,6 +98,9 @@ def load_library(path: Optional[str] = None):
     lib.fc_profile.argtypes = [vp, c_int]
     lib.fc_profile.restype = c_int
     lib.fc_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(c_int)]
+    lib.fc_profile_timeline.argtypes = [vp, c_int, i32p, ctypes.POINTER(ctypes.c_float),
+                                        ctypes.POINTER(ctypes.c_float), ctypes.POINTER(c_int)]
+    lib.fc_profile_timeline.restype = c_int
     lib.fc_profile_read.restype = c_int
     lib.fc_selftest_wait_timeout.argtypes = [vp, vp, c_int]
     lib.fc_selftest_wait_timeout.restype = c_int
@@ -264,6 +271,24 @@ class FlashCache:
             raise FlashCacheError(st, "fc_get_error")
         return int(w.value)
 
+    def set_qkv_kernel(self, which: str, split: int = 0) -> None:
+        """Projection kernel of the tensor-core path: "auto", "pair" or "splitk";
+        ``split`` forces the split-K cluster size (0: chosen by shape)."""
+        for opt, val in ((1, {"auto": 0, "pair": 1, "splitk": 2}[which]), (2, int(split))):
+            st = self.lib.fc_set_option(self._h, opt, val)
+            if st != 0:
+                raise FlashCacheError(st, "fc_set_option")
+
+    def qkv_plan(self, total_q: int) -> dict:
+        """The projection kernel fc_step launches for ``total_q`` query rows."""
+        k, sp, mc = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        st = self.lib.fc_qkv_plan(self._h, int(total_q), ctypes.byref(k), ctypes.byref(sp),
+                                  ctypes.byref(mc))
+        if st != 0:
+            raise FlashCacheError(st, "fc_qkv_plan")
+        return {"kernel": ("cuda_core", "pair", "splitk")[k.value], "split": sp.value,
+                "max_clusters": mc.value}
+
     def last_step_work(self):
         """(work items, items of the two-pass kernel, items handed over to it) of
         the last step; waits for the last stream used."""
@@ -287,6 +312,18 @@ class FlashCache:
         if st != 0:
             raise FlashCacheError(st, "fc_profile_read")
         return {name: (float(ms[i]), int(n[i])) for i, name in enumerate(PROFILE_SLOTS)}
+
+    def profile_timeline(self, max_records: int = 4096):
+        """[(kernel or copy slot, start ms, end ms)] of the records so far, times
+        after the first record's start; call before profile_read (which clears)."""
+        sl = (ctypes.c_int32 * max_records)()
+        a = (ctypes.c_float * max_records)()
+        b = (ctypes.c_float * max_records)()
+        n = ctypes.c_int(0)
+        st = self.lib.fc_profile_timeline(self._h, max_records, sl, a, b, ctypes.byref(n))
+        if st != 0:
+            raise FlashCacheError(st, "fc_profile_timeline")
+        return [(PROFILE_SLOTS[sl[i]], float(a[i]), float(b[i])) for i in range(n.value)]
 
     def selftest_wait_timeout(self, limit_us: int, stream=None) -> None:
         """Enqueue the bounded-wait self-test (see fc_selftest_wait_timeout)."""

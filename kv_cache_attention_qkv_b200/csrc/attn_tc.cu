@@ -644,7 +644,7 @@ cudaError_t launch_attn_tc(const fc_handle* h, cudaStream_t st, const StepShape&
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(attn_tc_kernel, dim3(h->num_sms), dim3(THREADS), smem, st, h->tm_q, tm_k, tm_v, p);
+  e = launch_pdl_if(h->pdl, attn_tc_kernel, dim3(h->num_sms), dim3(THREADS), smem, st, h->tm_q, tm_k, tm_v, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

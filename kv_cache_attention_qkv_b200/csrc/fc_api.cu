@@ -46,12 +46,14 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// Record-before / record-after around one launch when profiling is on.
+// Record-before / record-after around one launch when profiling is on; in a
+// pipelined host-buffer step, also a timed event on each side of the launch.
 struct ProfScope {
   fc_handle* h;
   cudaStream_t st;
   int idx = -1;
   ProfScope(fc_handle* h_, cudaStream_t st_, int slot) : h(h_), st(st_) {
+    fence();
     if (h->profiling && h->prof_n < 4096) {
       idx = h->prof_n++;
       h->prof_slot[idx] = slot;
@@ -60,6 +62,10 @@ struct ProfScope {
   }
   ~ProfScope() {
     if (idx >= 0) cudaEventRecord(h->prof_ev[2 * idx + 1], st);
+    fence();
+  }
+  void fence() {
+    if (h->hp.fencing) cudaEventRecord(h->hp.fence[h->hp.fence_i++ & 1u], st);
   }
 };
 
@@ -178,6 +184,8 @@ fc_status fc_create(const fc_config* cfg, const void* w_qkv, fc_handle** out) {
                         (H % 2) == 0;
   h->tc_gemm = tc_shape;
   h->tc_attn = tc_shape;
+  if (tc_shape)
+    for (int sp = 2; sp <= 8; ++sp) h->splitk_clusters[sp] = fc::qkv_splitk_max_clusters(sp);
 
   const int qtile = h->tc_attn ? fc::kTcQTile : fc::kSimtQTile;
   h->ws.max_items = H * (cfg->max_total_q / qtile + cfg->max_batch + 1);
@@ -249,6 +257,32 @@ fc_status fc_step(fc_handle* h, void* stream, int batch, const void* x, const in
 
 }  // extern "C"
 
+// Projection kernel of the tensor-core path for total_q query rows: the
+// CTA-pair kernel unless the split-K kernel is forced (FC_OPT_QKV_KERNEL).
+// The split-K kernel spreads each 128-row tile's reduction over a cluster of
+// `split` CTAs; measured on one B200 it was never faster than the pair kernel
+// (a 128 x 4096 query: 42.5 us at split 2 against 41.3 us, and 66-146 us at
+// splits 3-8, whose clusters no longer fit the GPU at once; hidden 256:
+// 27 against 19 us), so the default keeps the pair kernel.  With a split
+// forced, the largest split whose clusters all fit at once is the default
+// cluster size (at most 8 and one CTA per 64-wide K step).
+struct QkvPlan {
+  int kernel;  // 0 CUDA-core path, 1 CTA pair, 2 split-K
+  int split;
+};
+static QkvPlan plan_qkv(const fc_handle* h, int total_q) {
+  if (!h->tc_gemm) return {0, 0};
+  const fc_config& c = h->cfg;
+  const int n_tiles = 3 * c.n_heads * c.head_dim / 256;
+  const int tiles = (total_q + 127) / 128 * n_tiles;
+  const int smax = c.hidden / 64 < 8 ? c.hidden / 64 : 8;
+  if (h->qkv_kernel != 2) return {1, 0};
+  if (h->qkv_split > 0) return {2, h->qkv_split};
+  for (int sp = smax; sp >= 2; --sp)
+    if (tiles <= h->splitk_clusters[sp]) return {2, sp};
+  return {2, 1};
+}
+
 fc_status fc::step_impl(fc_handle* h, const CUtensorMap* tm_w, void* stream, int batch,
                         const void* x, const int32_t* q_pos,
                         const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int total_q,
@@ -294,8 +328,12 @@ fc_status fc::step_impl(fc_handle* h, const CUtensorMap* tm_w, void* stream, int
     if (!fc::encode_bf16_2d(&tm_x, x, (uint64_t)total_q, (uint64_t)c.hidden,
                             (uint64_t)c.hidden * 2, fc::kQkvXBoxRows, 64))
       return cuda_fail(h, -1, cudaErrorInvalidValue);
+    const QkvPlan plan = plan_qkv(h, total_q);
+    if (plan.kernel == 2 && plan.split > c.hidden / 64) return FC_ERR_INVALID_ARG;
     ProfScope ps(h, st, 1);
-    e = fc::launch_qkv_tc(h, st, s, tm_x, *tm_w, q_pos, k_cache, v_cache);
+    e = plan.kernel == 2
+            ? fc::launch_qkv_splitk(h, st, s, tm_x, *tm_w, q_pos, k_cache, v_cache, plan.split)
+            : fc::launch_qkv_tc(h, st, s, tm_x, *tm_w, q_pos, k_cache, v_cache);
   } else {
     ProfScope ps(h, st, 1);
     e = fc::launch_qkv_simt(h, st, s, x, q_pos, k_cache, v_cache);
@@ -399,13 +437,43 @@ fc_status fc_get_error(fc_handle* h, int32_t* device_error_word) {
 
 int fc_last_launch_count(const fc_handle* h) { return h ? h->last_launches : 0; }
 
+fc_status fc_qkv_plan(const fc_handle* h, int total_q, int* kernel, int* split,
+                      int* max_clusters) {
+  if (!h || total_q < 0 || !kernel || !split) return FC_ERR_INVALID_ARG;
+  const QkvPlan p = plan_qkv(h, total_q);
+  *kernel = p.kernel;
+  *split = p.split;
+  if (max_clusters) {
+    const int smax = h->cfg.hidden / 64 < 8 ? h->cfg.hidden / 64 : 8;
+    const int sp = p.split >= 2 ? p.split : smax;
+    *max_clusters = (h->tc_gemm && sp >= 2) ? h->splitk_clusters[sp] : 0;
+  }
+  return FC_OK;
+}
+
+fc_status fc_set_option(fc_handle* h, int option, int value) {
+  if (!h) return FC_ERR_INVALID_ARG;
+  if (option == FC_OPT_QKV_KERNEL) {
+    if (value < 0 || value > 2) return FC_ERR_INVALID_ARG;
+    h->qkv_kernel = value;
+    return FC_OK;
+  }
+  if (option == FC_OPT_QKV_SPLIT) {
+    if (value < 0 || value > 8) return FC_ERR_INVALID_ARG;
+    h->qkv_split = value;
+    return FC_OK;
+  }
+  return FC_ERR_INVALID_ARG;
+}
+
 const char* fc_last_cuda_error(const fc_handle* h) {
   static const char* const kSlot[] = {"prep", "qkv_rope_scatter", "attention",
-                                      "importance_finalize", "topk", "attention_one_pass"};
+                                      "importance_finalize", "topk", "attention_one_pass",
+                                      "h2d_copy", "d2h_copy"};
   static thread_local char buf[256];
   if (!h || h->last_cuda_err == cudaSuccess) return "no CUDA error recorded";
   snprintf(buf, sizeof(buf), "%s: %s (%s)",
-           h->last_cuda_slot >= 0 && h->last_cuda_slot < 6 ? kSlot[h->last_cuda_slot]
+           h->last_cuda_slot >= 0 && h->last_cuda_slot < 8 ? kSlot[h->last_cuda_slot]
                                                            : "host call",
            cudaGetErrorName(h->last_cuda_err), cudaGetErrorString(h->last_cuda_err));
   return buf;
@@ -432,6 +500,29 @@ fc_status fc_profile(fc_handle* h, int enable) {
       if (cudaEventCreate(&h->prof_ev[i]) != cudaSuccess) return FC_ERR_CUDA;
   }
   h->profiling = enable != 0;
+  return FC_OK;
+}
+
+fc_status fc_profile_timeline(fc_handle* h, int max_records, int32_t* slot, float* start_ms,
+                              float* end_ms, int* n) {
+  if (!h || max_records < 0 || !n || (max_records > 0 && (!slot || !start_ms || !end_ms)))
+    return FC_ERR_INVALID_ARG;
+  *n = 0;
+  if (!h->prof_ev || h->prof_n == 0) return FC_OK;
+  if (cudaSetDevice(h->device) != cudaSuccess) return FC_ERR_CUDA;
+  const int m = h->prof_n < max_records ? h->prof_n : max_records;
+  for (int i = 0; i < h->prof_n; ++i)
+    if (cudaEventSynchronize(h->prof_ev[2 * i + 1]) != cudaSuccess) return FC_ERR_CUDA;
+  for (int i = 0; i < m; ++i) {
+    float a = 0.f, b = 0.f;
+    if (cudaEventElapsedTime(&a, h->prof_ev[0], h->prof_ev[2 * i]) != cudaSuccess ||
+        cudaEventElapsedTime(&b, h->prof_ev[0], h->prof_ev[2 * i + 1]) != cudaSuccess)
+      return FC_ERR_CUDA;
+    slot[i] = h->prof_slot[i];
+    start_ms[i] = a;
+    end_ms[i] = b;
+  }
+  *n = m;
   return FC_OK;
 }
 

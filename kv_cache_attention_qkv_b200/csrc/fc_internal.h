@@ -101,6 +101,11 @@ struct HostPipe {
   int32_t* tracked[2] = {nullptr, nullptr};  // [max_batch, max_topk]
   float* importance = nullptr;            // [max_total_k]
   cudaEvent_t h2d_done[2] = {}, comp_done[2] = {}, d2h_done[2] = {};
+  // timed events recorded around each kernel of a pipelined step (never
+  // queried; see fc_step_host)
+  cudaEvent_t fence[2] = {};
+  unsigned fence_i = 0;
+  bool fencing = false;
   unsigned long long calls = 0;
 };
 }  // namespace fc
@@ -116,6 +121,16 @@ struct fc_handle {
   fc::Workspace ws;
   cudaStream_t last_stream = nullptr;
   int last_launches = 0;
+  // launch the step's kernels with programmatic dependent launch (off while
+  // fc_step_host runs: between the copies of neighbouring steps it lengthened
+  // the pipelined step by a quarter)
+  bool pdl = true;
+  // projection kernel on the tensor-core path: 0 chooses by shape, 1 the CTA
+  // pair kernel, 2 the split-K cluster kernel (fc_set_option)
+  int qkv_kernel = 0;
+  int qkv_split = 0;  // split-K cluster size: 0 chosen by shape, else forced
+  // resident clusters of the split-K projection kernel per cluster size 2..8
+  int splitk_clusters[9] = {};
   // the last CUDA call of fc_step that failed: its error and the profile slot
   // of the kernel being launched (-1: not a launch)
   cudaError_t last_cuda_err = cudaSuccess;
@@ -132,16 +147,30 @@ struct fc_handle {
 
 namespace fc {
 void free_host_pipe(fc_handle* h);
+
+// Begin / end one profiling record (slot, event pair) on a stream; no-op
+// unless fc_profile is on.  Returns the record index or -1.
+inline int prof_begin(fc_handle* h, cudaStream_t st, int slot) {
+  if (!h->profiling || h->prof_n >= 4096) return -1;
+  const int idx = h->prof_n++;
+  h->prof_slot[idx] = slot;
+  cudaEventRecord(h->prof_ev[2 * idx], st);
+  return idx;
+}
+inline void prof_end(fc_handle* h, cudaStream_t st, int idx) {
+  if (idx >= 0) cudaEventRecord(h->prof_ev[2 * idx + 1], st);
+}
 }
 
 namespace fc {
 
-// Launch with programmatic stream serialisation: the kernel may be scheduled
-// while the previous kernel of the stream is still running; it must call
-// griddepcontrol.wait before touching that kernel's outputs.
+// Launch with programmatic stream serialisation (when `pdl`): the kernel may
+// be scheduled while the previous kernel of the stream is still running; it
+// must call griddepcontrol.wait before touching that kernel's outputs (a
+// no-op when it was launched without the attribute).
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t st, Args... args) {
+cudaError_t launch_pdl_if(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t st, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -151,8 +180,14 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  return launch_pdl_if(true, kernel, grid, block, smem, st, args...);
 }
 
 // ---- launchers (each returns the CUDA error of its launch) -----------------
@@ -167,6 +202,14 @@ cudaError_t launch_attn_simt(const fc_handle* h, cudaStream_t st, const StepShap
 cudaError_t launch_qkv_tc(const fc_handle* h, cudaStream_t st, const StepShape& s,
                           const CUtensorMap& tm_x, const CUtensorMap& tm_w, const int32_t* q_pos,
                           void* k_cache, void* v_cache);
+cudaError_t launch_qkv_splitk(const fc_handle* h, cudaStream_t st, const StepShape& s,
+                              const CUtensorMap& tm_x, const CUtensorMap& tm_w,
+                              const int32_t* q_pos, void* k_cache, void* v_cache, int split);
+size_t qkv_splitk_smem_bytes();
+// thread-block clusters of `split` CTAs of the split-K kernel that can be
+// resident at once (cudaOccupancyMaxActiveClusters); minus the CUDA error
+// code when the query fails
+int qkv_splitk_max_clusters(int split);
 cudaError_t launch_gemm_tc(int num_sms, cudaStream_t st, const CUtensorMap& tm_a,
                            const CUtensorMap& tm_b0, const CUtensorMap& tm_b1, GemmParams p);
 size_t gemm_tc_smem_bytes();

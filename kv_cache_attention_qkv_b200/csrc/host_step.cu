@@ -55,7 +55,8 @@ fc_status init_pipe(fc_handle* h) {
          cudaMalloc(&p.tracked[s], (size_t)c.max_batch * topk * sizeof(int32_t)) == cudaSuccess &&
          cudaEventCreateWithFlags(&p.h2d_done[s], cudaEventDisableTiming) == cudaSuccess &&
          cudaEventCreateWithFlags(&p.comp_done[s], cudaEventDisableTiming) == cudaSuccess &&
-         cudaEventCreateWithFlags(&p.d2h_done[s], cudaEventDisableTiming) == cudaSuccess;
+         cudaEventCreateWithFlags(&p.d2h_done[s], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreate(&p.fence[s]) == cudaSuccess;
   }
   if (!ok) {
     const cudaError_t e = cudaGetLastError();
@@ -81,6 +82,7 @@ void free_host_pipe(fc_handle* h) {
     if (p.h2d_done[s]) cudaEventDestroy(p.h2d_done[s]);
     if (p.comp_done[s]) cudaEventDestroy(p.comp_done[s]);
     if (p.d2h_done[s]) cudaEventDestroy(p.d2h_done[s]);
+    if (p.fence[s]) cudaEventDestroy(p.fence[s]);
   }
   if (p.importance) cudaFree(p.importance);
   if (p.s_h2d) cudaStreamDestroy(p.s_h2d);
@@ -122,6 +124,7 @@ fc_status fc_step_host(fc_handle* h, void* stream, int batch, const void* x, con
   // ---- inputs: host -> staging set s, once call n-2's kernels are done with it
   cudaError_t e = cudaSuccess;
   if (reuse) e = cudaStreamWaitEvent(p.s_h2d, p.comp_done[s], 0);
+  const int rec_in = fc::prof_begin(h, p.s_h2d, 6);
   auto h2d = [&](void* dst, const void* src, size_t bytes) {
     if (e == cudaSuccess && bytes > 0)
       e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, p.s_h2d);
@@ -133,26 +136,41 @@ fc_status fc_step_host(fc_handle* h, void* stream, int batch, const void* x, con
   h2d(sm + L.lo, cand_lo, (size_t)batch * sizeof(int32_t));
   h2d(sm + L.hi, cand_hi, (size_t)batch * sizeof(int32_t));
   if (k_per_seq) h2d(sm + L.kps, k_per_seq, (size_t)batch * sizeof(int32_t));
+  fc::prof_end(h, p.s_h2d, rec_in);
   if (e == cudaSuccess) e = cudaEventRecord(p.h2d_done[s], p.s_h2d);
   // ---- kernels on the caller's stream
   if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, p.h2d_done[s], 0);
   if (e == cudaSuccess && reuse) e = cudaStreamWaitEvent(cs, p.d2h_done[s], 0);
   if (e != cudaSuccess) return FC_ERR_CUDA;
+  // The kernels run here beside the input copy of the next call and the
+  // output copy of the previous one.  Launched back to back they stretched
+  // the input copy (batch 32 x 128 rows, 33.5 MB: 1.05 ms at 32 GB/s instead
+  // of 0.75 ms at 44 GB/s) and the step to 1.0-1.05 ms; with a timed event
+  // recorded on each side of every kernel (which also ends programmatic
+  // overlap between them, so the kernels are launched plainly) the step takes
+  // 0.77-0.80 ms, near the two copies' concurrent rate.  Timing-disabled
+  // events, or timed events around a single kernel, did not help.
+  h->pdl = false;
+  p.fencing = true;
   st = fc_step(h, stream, batch, p.x[s], sm + L.q_pos, sm + L.cu_q, sm + L.cu_k, total_q, total_k,
                k_cache, v_cache, p.out[s], p.importance, 0);
-  if (st != FC_OK) return st;
   const int step_launches = h->last_launches;
-  st = fc_topk_tracked(h, stream, batch, total_k, p.importance, sm + L.cu_k, sm + L.lo, sm + L.hi,
-                       k_per_seq ? sm + L.kps : nullptr, k, p.tracked[s]);
+  if (st == FC_OK)
+    st = fc_topk_tracked(h, stream, batch, total_k, p.importance, sm + L.cu_k, sm + L.lo, sm + L.hi,
+                         k_per_seq ? sm + L.kps : nullptr, k, p.tracked[s]);
+  h->pdl = true;
+  p.fencing = false;
   if (st != FC_OK) return st;
   h->last_launches += step_launches;
   e = cudaEventRecord(p.comp_done[s], cs);
   // ---- outputs: staging set s -> host
   if (e == cudaSuccess) e = cudaStreamWaitEvent(p.s_d2h, p.comp_done[s], 0);
+  const int rec_out = fc::prof_begin(h, p.s_d2h, 7);
   if (e == cudaSuccess && out_bytes > 0)
     e = cudaMemcpyAsync(out, p.out[s], out_bytes, cudaMemcpyDeviceToHost, p.s_d2h);
   if (e == cudaSuccess && tr_bytes > 0)
     e = cudaMemcpyAsync(tracked, p.tracked[s], tr_bytes, cudaMemcpyDeviceToHost, p.s_d2h);
+  fc::prof_end(h, p.s_d2h, rec_out);
   if (e == cudaSuccess) e = cudaEventRecord(p.d2h_done[s], p.s_d2h);
   if (e != cudaSuccess) return FC_ERR_CUDA;
   ++p.calls;

@@ -384,7 +384,7 @@ cudaError_t launch_qkv_tc(const fc_handle* h, cudaStream_t st, const StepShape& 
   int max_clusters = 0;
   cfg.numAttrs = 1;  // occupancy query with the cluster shape only
   const bool occ_ok = cudaOccupancyMaxActiveClusters(&max_clusters, qkv_tc_kernel, &cfg) == cudaSuccess;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = h->pdl ? 2 : 1;
   if (occ_ok &&
       max_clusters > 0 && max_clusters < pairs) {
     pairs = max_clusters;

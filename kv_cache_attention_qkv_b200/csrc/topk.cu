@@ -193,7 +193,7 @@ cudaError_t launch_importance_finalize(const fc_handle* h, cudaStream_t st, int 
   if (S <= 0) return cudaSuccess;
   int blocks = (S + 255) / 256;
   if (blocks > h->num_sms * 8) blocks = h->num_sms * 8;
-  cudaError_t e = launch_pdl(importance_finalize, dim3(blocks), dim3(256), 0, st, S, h->ws.imp_acc,
+  cudaError_t e = launch_pdl_if(h->pdl, importance_finalize, dim3(blocks), dim3(256), 0, st, S, h->ws.imp_acc,
                              importance, accumulate);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -202,7 +202,7 @@ cudaError_t launch_importance_finalize(const fc_handle* h, cudaStream_t st, int 
 cudaError_t launch_topk(const fc_handle* h, cudaStream_t st, int B, int S, const float* importance,
                         const int32_t* cu_k, const int32_t* cand_lo, const int32_t* cand_hi,
                         const int32_t* k_per_seq, int k, int32_t* tracked) {
-  cudaError_t e = launch_pdl(topk_kernel, dim3(B), dim3(TK_THREADS), 0, st, B, importance, cu_k,
+  cudaError_t e = launch_pdl_if(h->pdl, topk_kernel, dim3(B), dim3(TK_THREADS), 0, st, B, importance, cu_k,
                              cand_lo, cand_hi, k_per_seq, k, tracked, h->ws.err, S, h->cfg.max_pos);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

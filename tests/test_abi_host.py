@@ -85,6 +85,7 @@ def test_calls_on_a_null_handle_are_rejected(lib):
     w = ctypes.c_int32()
     assert lib.fc_get_error(None, ctypes.byref(w)) == -1
     assert lib.fc_last_launch_count(None) == 0
+    assert lib.fc_set_option(None, 1, 0) == -1
     lib.fc_destroy(None)  # no-op
 
 

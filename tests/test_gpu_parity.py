@@ -29,6 +29,37 @@ def test_full_parity(name):
     tl.assert_close(gpu["importance"], ref["importance"], tl.TOL[inp.dtype], "importance")
 
 
+@pytest.mark.parametrize("name", ["layer_b1", "small_varlen", "small_longcache"])
+def test_both_projection_kernels(name):
+    """The CTA-pair projection and the split-K cluster projection (forced, at
+    several cluster sizes) all meet the parity bar on every output, and the
+    default run is bit-identical to a forced run of the kernel it planned."""
+    inp = workloads.generate(name)
+    ref = tl.run_oracle(inp)
+    outs = {}
+    smax = min(8, inp.hidden // 64)
+    for which, split in (("pair", 0), ("splitk", 0), ("splitk", 1), ("splitk", 2),
+                         ("splitk", smax), ("auto", 0)):
+        dev = tl.upload(inp)
+        layer = tl.make_layer(inp, dev["w"])
+        layer.set_qkv_kernel(which, split)
+        plan = layer.qkv_plan(inp.total_q)
+        gpu = tl.run_gpu(inp, layer=layer, dev=dev)
+        assert gpu["err"] == 0, (which, split)
+        tl.compare_step(inp, gpu, ref, range(inp.batch))
+        tl.assert_unwritten_rows_unchanged(inp, gpu)
+        outs[(which, split)] = (plan, gpu["out"], dev["k_cache"].cpu(), dev["v_cache"].cpu())
+    # the default run is bit-identical to the forced run of the kernel it planned
+    auto = outs[("auto", 0)]
+    if auto[0]["kernel"] == "pair":
+        same = outs[("pair", 0)]
+    else:
+        same = next(v for (w, sp), v in outs.items()
+                    if w == "splitk" and v[0]["split"] == auto[0]["split"])
+    assert np.array_equal(auto[1], same[1])
+    assert torch.equal(auto[2], same[2]) and torch.equal(auto[3], same[3])
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("name,seqs", [("batch32_uniform", [0, 13, 31]),
                                        ("batch32_varlen", [0, 5, 17, 30]),
