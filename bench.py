@@ -274,11 +274,16 @@ def _step_result(args, inp, ws, *, total_ms, burst_ms, per_kernel, launches, err
     T = inp.total_q
     # a step with importance runs the two-pass attention kernel alone; a step
     # without runs the one-pass kernel and the two-pass kernel for the items it
-    # hands over (usually none): its attention is the sum of the two
+    # hands over (usually none): its attention is the sum of the two.  A small
+    # batch split over the SMs runs two launches (row statistics, then pass 2
+    # and the combine): its attention is their sum too.
     per_kernel = dict(per_kernel)
-    if getattr(args, "no_importance", False) and "attention_one_pass" in per_kernel:
+    if getattr(args, "no_importance", False) and per_kernel.get("attention_one_pass", (0, 0))[1]:
         (ma, na), (mb, _) = per_kernel["attention_one_pass"], per_kernel["attention"]
         per_kernel["attention"] = (ma + mb, na)
+    if per_kernel.get("attention_split_pass1", (0, 0))[1]:
+        (ma, _), (mb, nb) = per_kernel["attention_split_pass1"], per_kernel["attention"]
+        per_kernel["attention"] = (ma + mb, nb)
     ms_per_step = total_ms / args.steps
     tokens = T * ws * args.steps
     value = tokens / (total_ms / 1e3)
@@ -363,6 +368,7 @@ def run_ours(args):
                        max_seqlen_q=int(np.diff(inp.cu_seqlens_q).max()),
                        max_pos=int(np.diff(inp.cu_seqlens_k).max()), max_topk=K)
     layer.set_qkv_kernel(args.qkv_kernel, args.qkv_split)
+    layer.set_attn_split({"auto": True, "never": False, "always": "always"}[args.attn_split])
     out = torch.empty((T, H, d), device=dev, dtype=dt)
     imp = torch.empty((S,), device=dev, dtype=torch.float32)
     tracked = torch.empty((B, K), device=dev, dtype=torch.int32)
@@ -940,6 +946,9 @@ def main():
                     help="projection kernel of the tensor-core path (default: the CTA-pair kernel)")
     ap.add_argument("--qkv-split", type=int, default=0,
                     help="cluster size of the split-K projection (default: the largest that fits at once)")
+    ap.add_argument("--attn-split", choices=["auto", "never", "always"], default="auto",
+                    help="small-batch attention split over the SMs (default: small batches "
+                         "with caches of 2048 rows or more)")
     ap.add_argument("--sweep", choices=sorted(SWEEPS) + ["all"], default=None,
                     help="time every point of a sweep axis (one JSON line per point, no cpu_baseline)")
     args = ap.parse_args()

@@ -269,10 +269,23 @@ FC_API const char* fc_last_cuda_error(const fc_handle* h);
  *     cut into that many nearly equal runs of 64-wide steps; a value above
  *     hidden / 64 leaves some CTAs without a step and is rejected at fc_step
  *     with FC_ERR_INVALID_ARG.
+ *   FC_OPT_ATTN_SPLIT: small-batch attention on the tensor-core path.  0
+ *     (default): when H * (ceil(total_q / 128) + batch - 1) is at most the
+ *     SM count and the caches hold 2048 rows or more on average
+ *     (total_k >= 2048 * batch), every (sequence, head, 128-row query tile)
+ *     item is split into max(1, min(SMs / items, 8, its 128-key tiles / 4))
+ *     entries over runs of key tiles (at least four tiles each); a first launch stores each entry's row
+ *     maxima and normalisers, a second combines them into the rows'
+ *     log-sum-exp, computes P, P V and the column sums over its own keys, and
+ *     the item's last entry adds the parts of O in entry order (so results do
+ *     not depend on timing).  1: never split.  2: split whenever the batch is
+ *     small enough, whatever the cache length, down to one tile per entry
+ *     (for tests and measurement).
  * FC_ERR_INVALID_ARG for an unknown option or value.
  */
 #define FC_OPT_QKV_KERNEL 1
 #define FC_OPT_QKV_SPLIT 2
+#define FC_OPT_ATTN_SPLIT 3
 FC_API fc_status fc_set_option(fc_handle* h, int option, int value);
 
 /*
@@ -306,9 +319,12 @@ FC_API int fc_last_launch_count(const fc_handle* h);
  * fc_profile_read waits for the recorded work, writes for each slot
  * (0 prep, 1 qkv_rope_scatter, 2 attention (the two-pass attention kernel
  * of the tensor-core path: every item of a step with importance, the items
- * handed over in a step without), 3 importance_finalize, 4 topk,
- * 5 attention_one_pass (the one-pass kernel of a tensor-core step without
- * importance), 6 h2d_copy and 7 d2h_copy (the copy blocks of fc_step_host))
+ * handed over in a step without; in a small-batch step whose items are split
+ * over the SMs, its second launch: pass 2 and the combine of the parts),
+ * 3 importance_finalize, 4 topk, 5 attention_one_pass (the one-pass kernel of
+ * a tensor-core step without importance), 6 h2d_copy and 7 d2h_copy (the copy
+ * blocks of fc_step_host), 8 attention_split_pass1 (the first launch of a
+ * split small-batch step: every entry's row statistics))
  * the summed milliseconds to ms[slot] and the record count to launches[slot]
  * (host arrays of FC_PROFILE_SLOTS entries), and clears the records.
  * fc_profile_timeline (call it before fc_profile_read) waits for the recorded
@@ -316,7 +332,7 @@ FC_API int fc_last_launch_count(const fc_handle* h);
  * order, the slot and the start and end times in milliseconds after the first
  * record's start (host arrays); *n receives the number written.
  */
-#define FC_PROFILE_SLOTS 8
+#define FC_PROFILE_SLOTS 9
 FC_API fc_status fc_profile(fc_handle* h, int enable);
 FC_API fc_status fc_profile_timeline(fc_handle* h, int max_records, int32_t* slot, float* start_ms,
                                      float* end_ms, int* n);

@@ -29,7 +29,7 @@ EXPORTED = ("fc_create", "fc_step", "fc_topk_tracked", "fc_step_host", "fc_host_
             "fc_decode_iteration", "fc_model_lm_head", "fc_last_step_work",
             "fc_last_cuda_error", "fc_profile_timeline", "fc_set_option", "fc_qkv_plan")
 PROFILE_SLOTS = ("prep", "qkv_rope_scatter", "attention", "importance_finalize", "topk",
-                 "attention_one_pass", "h2d_copy", "d2h_copy")
+                 "attention_one_pass", "h2d_copy", "d2h_copy", "attention_split_pass1")
 
 
 class FlashCacheError(RuntimeError):
@@ -278,6 +278,14 @@ class FlashCache:
             st = self.lib.fc_set_option(self._h, opt, val)
             if st != 0:
                 raise FlashCacheError(st, "fc_set_option")
+
+    def set_attn_split(self, mode) -> None:
+        """Small-batch attention split: True/"auto" (default: small batches with
+        long caches), False/"never", or "always" (any cache length)."""
+        val = {True: 0, "auto": 0, False: 1, "never": 1, "always": 2}[mode]
+        st = self.lib.fc_set_option(self._h, 3, val)
+        if st != 0:
+            raise FlashCacheError(st, "fc_set_option")
 
     def qkv_plan(self, total_q: int) -> dict:
         """The projection kernel fc_step launches for ``total_q`` query rows."""

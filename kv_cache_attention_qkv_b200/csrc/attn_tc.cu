@@ -28,6 +28,16 @@
 // 64h..64h+63 of a tile go, packed, to columns 64h..64h+31 of its buffer: every
 // softmax warp overwrites only columns it has already read itself.
 //
+// Small batches (too few items to fill the SMs) split each item's cache
+// across several work entries of the list (key tiles [j0, j1) each) and run
+// the two passes as two launches of this kernel: mode 1 stores every entry's
+// per-row (max, normaliser) over its key tiles; mode 2 combines the entries'
+// statistics of the item into the row's log-sum-exp, runs pass 2 over its
+// own tiles (column sums are complete, every key belongs to one entry) and
+// stores its part of O (already normalised, fp32); the entry that finishes
+// last sums the parts in entry order and writes the output, so the result
+// does not depend on which CTA finishes first.  Mode 0 is the fused kernel.
+//
 // TMEM columns: S/P buffer 0 [0,128), S/P buffer 1 [128,256), O [256,384),
 // Q [384,448).
 //
@@ -89,6 +99,10 @@ struct AttnParams {
   __nv_bfloat16* out;
   unsigned long long* imp_acc;
   int want_imp;
+  float* stats;  // [entry][m, l][128] row statistics of the entries (modes 1, 2)
+  float* opart;  // [entry][128][128] fp32 parts of O of split items (mode 2)
+  int32_t* gcnt; // [first entry of an item] entries of the item done (mode 2)
+  int max_entries;
   int32_t* err;
 };
 
@@ -99,13 +113,16 @@ struct __align__(8) AttnBars {
   unsigned long long pready[2];
   unsigned long long ofull, ofree;
   unsigned long long statbar;
+  unsigned long long obar, obar2;  // split items: parts of O stored / last-entry flag set
   unsigned long long drain;
   uint32_t tmem_base;
   int abort_flag;
 };
 
 struct Item {
-  int b, qt, h, q0, nrows, k0, L, ntiles;
+  int b, qt, h, q0, nrows, k0, L;
+  int j0, j1;     // this entry's key tiles
+  int first, ns;  // the item's first entry in the list and its entry count
 };
 
 __device__ __forceinline__ Item to_item(const WorkItem& w) {
@@ -117,7 +134,10 @@ __device__ __forceinline__ Item to_item(const WorkItem& w) {
   r.nrows = w.nrows;
   r.k0 = w.k0;
   r.L = w.L;
-  r.ntiles = (r.L + KT - 1) / KT;
+  r.j0 = (int)((unsigned)w.pad[0] & 0xFFFFu);
+  r.j1 = (int)((unsigned)w.pad[0] >> 16);
+  r.first = (int)((unsigned)w.pad[1] & 0x0FFFFFFFu);
+  r.ns = (int)((unsigned)w.pad[1] >> 28);
   return r;
 }
 
@@ -165,6 +185,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, AttnParams p) {
@@ -197,6 +218,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     ptx::mbar_init(bar(bars->ofull), 1);
     ptx::mbar_init(bar(bars->ofree), SOFTMAX_WARPS);
     ptx::mbar_init(bar(bars->statbar), SOFTMAX_WARPS);
+    ptx::mbar_init(bar(bars->obar), SOFTMAX_WARPS);
+    ptx::mbar_init(bar(bars->obar2), 1);
     ptx::mbar_init(bar(bars->drain), 1);
     bars->abort_flag = 0;
     ptx::fence_mbar_init();
@@ -255,14 +278,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         ptx::tma_load_2d(base + OFF_Q, &tm_q, 0, qrow, bar(bars->qfull));
         ptx::tma_load_2d(base + OFF_Q + HALF_BYTES, &tm_q, 64, qrow, bar(bars->qfull));
         q_issued_phase = (int)(ic & 1u);
-        for (int j = 0; j < t.ntiles && !failed; ++j) {
-          if (!load_tile(&tm_k, t.h, t.k0 + j * KT, pol_keep)) failed = true;
-        }
-        for (int j = 0; j < t.ntiles && !failed; ++j) {
-          if (!load_tile(&tm_k, t.h, t.k0 + j * KT, pol_stream) ||
-              !load_tile(&tm_v, t.h, t.k0 + j * KT, pol_stream))
-            failed = true;
-        }
+        if (MODE != 2)
+          for (int j = t.j0; j < t.j1 && !failed; ++j) {
+            if (!load_tile(&tm_k, t.h, t.k0 + j * KT, pol_keep)) failed = true;
+          }
+        if (MODE != 1)
+          for (int j = t.j0; j < t.j1 && !failed; ++j) {
+            if (!load_tile(&tm_k, t.h, t.k0 + j * KT, pol_stream) ||
+                !load_tile(&tm_v, t.h, t.k0 + j * KT, pol_stream))
+              failed = true;
+          }
       }
       if (failed) {
         *abort_flag = 1;
@@ -347,11 +372,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                                 ptx::smem_desc(q_addr + off, 16, 1024));
         }
         ptx::mma_commit(bar(bars->qfree));  // the shared-memory copy of Q is free again
+        const int nt = t.j1 - t.j0;
         // pass 1: S tiles only
-        for (int j = 0; j < t.ntiles && !failed; ++j)
-          if (!issue_s(cons + (uint32_t)j)) failed = true;
+        if (MODE != 2)
+          for (int j = 0; j < nt && !failed; ++j)
+            if (!issue_s(cons + (uint32_t)j)) failed = true;
         if (failed) break;
-        const uint32_t base2 = cons + (uint32_t)t.ntiles;
+        const uint32_t base2 = cons + (MODE != 2 ? (uint32_t)nt : 0u);
+        if (MODE == 1) {
+          cons = base2;
+          continue;
+        }
         const uint32_t sb0 = scnt & 1u;  // buffer of pass-2 tile 0
         // the previous item's O must have been read out before P V overwrites it
         if (!ptx::mbar_wait(bar(bars->ofree), (ic & 1u) ^ 1u, abort_flag)) {
@@ -360,19 +391,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         // S runs two tiles ahead of P V; S[j+2] reuses tile j's buffer and is
         // queued right after P V [j], which reads P[j] from that buffer
-        const int lead = t.ntiles < 2 ? t.ntiles : 2;
+        const int lead = nt < 2 ? nt : 2;
         for (int j = 0; j < lead && !failed; ++j)
           if (!issue_s(base2 + 2u * (uint32_t)j)) failed = true;
-        for (int j = 0; j < t.ntiles && !failed; ++j) {
+        for (int j = 0; j < nt && !failed; ++j) {
           if (!issue_pv(base2 + 2u * (uint32_t)j + 1u, (sb0 + (uint32_t)j) & 1u, j == 0)) {
             failed = true;
             break;
           }
-          if (j + 2 < t.ntiles && !issue_s(base2 + 2u * (uint32_t)(j + 2))) failed = true;
+          if (j + 2 < nt && !issue_s(base2 + 2u * (uint32_t)(j + 2))) failed = true;
         }
         if (failed) break;
         ptx::mma_commit(bar(bars->ofull));
-        cons = base2 + 2u * (uint32_t)t.ntiles;
+        cons = base2 + 2u * (uint32_t)nt;
       }
       if (failed) {
         *abort_flag = 1;
@@ -399,6 +430,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         reinterpret_cast<unsigned long long*>(smem + OFF_CSACC) + grp * 256 + col0;
     int* cnt_base = reinterpret_cast<int*>(smem + OFF_CSCNT) + grp * 4 + hf;
     uint32_t gs = 0, ic = 0;  // global S tile index (same sequence as the MMA warp)
+    uint32_t oc = 0;          // split items finished (obar / obar2 phases)
 
     // This thread's 64 columns of S tile `s` (buffer grp); the buffer is
     // released to the MMA warp at once.
@@ -434,7 +466,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     // the next item's record, field `lane` in lane `lane` (one register)
     auto fetch_field = [&](int it) -> int {
-      return (lane < 6 && it < n_items)
+      return (lane < 8 && it < n_items)
                  ? __ldg(reinterpret_cast<const int*>(item_ptr(p, n_long, it)) + lane)
                  : 0;
     };
@@ -448,18 +480,24 @@ __global__ void __launch_bounds__(THREADS, 1)
       wcur.nrows = __shfl_sync(0xffffffffu, fnext, 3);
       wcur.k0 = __shfl_sync(0xffffffffu, fnext, 4);
       wcur.L = __shfl_sync(0xffffffffu, fnext, 5);
+      wcur.pad[0] = __shfl_sync(0xffffffffu, fnext, 6);
+      wcur.pad[1] = __shfl_sync(0xffffffffu, fnext, 7);
       const Item t = to_item(wcur);
       fnext = fetch_field(snake_item(r + 1, blockIdx.x, gridDim.x));
       uint32_t sv[64];
+      const int nt = t.j1 - t.j0;
+      float M = -INFINITY, Ls = 0.f;  // the row's maximum and normaliser (all its keys)
+      if (MODE != 2) {
       // ---- pass 1: max and normaliser over this warp's tiles and column half
       float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < t.ntiles; ++j) {
-        const uint32_t s = gs + (uint32_t)j;
+      for (int jj = 0; jj < nt; ++jj) {
+        const uint32_t s = gs + (uint32_t)jj;
         if ((int)(s & 1u) != grp) continue;
         if (!load_s(s, sv)) {
           failed = true;
           break;
         }
+        const int j = t.j0 + jj;
         const int kmax = t.L - j * KT - col0;  // columns >= kmax are outside the sequence
         if (kmax <= 0) continue;
         float x[64];
@@ -481,7 +519,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         m = mn;
       }
       if (failed) break;
-      gs += (uint32_t)t.ntiles;
+      gs += (uint32_t)nt;
       // merge the four (group, half) parts of every row once per item
       float* st_par = stat + (ic & 1u) * (PARTS * 256);
       st_par[part * 256 + rl] = m;
@@ -492,22 +530,46 @@ __global__ void __launch_bounds__(THREADS, 1)
         failed = true;
         break;
       }
-      float M = -INFINITY;
 #pragma unroll
       for (int q = 0; q < PARTS; ++q) M = fmaxf(M, st_par[q * 256 + rl]);
-      float Ls = 0.f;
 #pragma unroll
       for (int q = 0; q < PARTS; ++q) {
         const float mq = st_par[q * 256 + rl];
         if (mq != -INFINITY) Ls += st_par[q * 256 + 128 + rl] * ex2(mq - M);
       }
+      if (MODE == 1) {  // this entry's statistics for the pass-2 launch
+        const int entry = it;
+        if (part == 0 && entry < p.max_entries) {
+          p.stats[(size_t)entry * 256 + rl] = M;
+          p.stats[(size_t)entry * 256 + 128 + rl] = Ls;
+        }
+        continue;
+      }
+      } else {
+        // the statistics of the item's entries (stored by the mode-1 launch),
+        // all loaded before they are combined in entry order
+        float me[8], le[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int entry = t.first + e;
+          const bool ok = e < t.ns && entry < p.max_entries;
+          me[e] = ok ? __ldcg(p.stats + (size_t)entry * 256 + rl) : -INFINITY;
+          le[e] = ok ? __ldcg(p.stats + (size_t)entry * 256 + 128 + rl) : 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) M = fmaxf(M, me[e]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (me[e] != -INFINITY) Ls += le[e] * ex2(me[e] - M);
+      }
       // rows past the query tile's end get lse = +inf, i.e. P = 0
       const float lse = rl < t.nrows ? M + __log2f(Ls) : INFINITY;
       // ---- pass 2: final probabilities -> P (TMEM, over its S tile); column sums
-      for (int j = 0; j < t.ntiles; ++j) {
-        const uint32_t s = gs + (uint32_t)j;
+      for (int jj = 0; jj < nt; ++jj) {
+        const uint32_t s = gs + (uint32_t)jj;
         if ((int)(s & 1u) != grp) continue;
         const uint32_t scol = sbuf + lane_off + (uint32_t)col0;
+        const int j = t.j0 + jj;
         const int kmax = t.L - j * KT - col0;  // columns >= kmax are outside the sequence
         if (!ptx::mbar_wait(bar(bars->sfull[grp]), (s >> 1) & 1u, abort_flag)) {
           failed = true;
@@ -581,7 +643,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       if (failed) break;
-      gs += (uint32_t)t.ntiles;
+      gs += (uint32_t)nt;
       // ---- O (already normalised) -> out: warp sw takes columns 32*(sw/4)..+31
       if (!ptx::mbar_wait(bar(bars->ofull), ic & 1u, abort_flag)) {
         failed = true;
@@ -594,6 +656,65 @@ __global__ void __launch_bounds__(THREADS, 1)
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(bars->ofree));
+      if (MODE == 2 && t.ns > 1) {
+        // a split item: store this entry's part; the item's last entry to
+        // finish adds the parts in entry order and writes the output
+        // layout [entry][column][row]: a warp's 32 rows of one column are
+        // 128 contiguous bytes
+        const int entry = it;
+        const bool in_ws = entry < p.max_entries && t.first + t.ns <= p.max_entries;
+        auto part_at = [&](int e) { return p.opart + ((size_t)e * HD + ocol) * QT + rl; };
+        if (rl < t.nrows && in_ws) {
+          float* op = part_at(entry);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) __stcg(op + c * QT, __uint_as_float(sv[c]));
+        }
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(bars->obar));
+        volatile int* last_flag = reinterpret_cast<volatile int*>(smem + OFF_CSCNT) + 8;
+        if (sw == 0 && lane == 0) {
+          int last = 0;
+          if (ptx::mbar_wait(bar(bars->obar), oc & 1u, abort_flag)) {
+            __threadfence();
+            if (in_ws) last = atomicAdd(&p.gcnt[t.first], 1) == t.ns - 1;
+            __threadfence();
+          } else {
+            *abort_flag = 1;
+          }
+          *last_flag = last;
+          ptx::mbar_arrive(bar(bars->obar2));
+        }
+        if (!ptx::mbar_wait(bar(bars->obar2), oc & 1u, abort_flag)) {
+          failed = true;
+          break;
+        }
+        ++oc;
+        if (*last_flag) {
+          __threadfence();
+          if (rl < t.nrows) {
+            // parts in entry order; this entry's own part from its registers
+            float acc[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+            for (int e = t.first; e < t.first + t.ns; ++e) {
+              if (e == entry) {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) acc[c] += __uint_as_float(sv[c]);
+              } else {
+                const float* src = part_at(e);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) acc[c] += __ldcg(src + c * QT);
+              }
+            }
+#pragma unroll
+            for (int c = 0; c < 32; ++c) sv[c] = __float_as_uint(acc[c]);
+          }
+          if (sw == 0 && lane == 0) p.gcnt[t.first] = 0;  // for the next launch
+        } else {
+          continue;
+        }
+      }
       if (rl < t.nrows) {
         uint4* dst = reinterpret_cast<uint4*>(
             p.out + ((size_t)(t.q0 + t.qt * QT + rl) * p.H + t.h) * HD + ocol);
@@ -626,7 +747,7 @@ size_t attn_tc_smem_bytes() { return OFF_BARS + sizeof(AttnBars) + 1024; }
 cudaError_t launch_attn_tc(const fc_handle* h, cudaStream_t st, const StepShape& s,
                            const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                            const int32_t* cu_q, const int32_t* cu_k, void* out,
-                           bool want_importance) {
+                           bool want_importance, int mode) {
   AttnParams p;
   p.H = s.H;
   p.max_T = h->cfg.max_total_q;
@@ -639,12 +760,18 @@ cudaError_t launch_attn_tc(const fc_handle* h, cudaStream_t st, const StepShape&
   p.out = (__nv_bfloat16*)out;
   p.imp_acc = h->ws.imp_acc;
   p.want_imp = want_importance ? 1 : 0;
+  p.stats = h->ws.split_stats;
+  p.opart = h->ws.split_o;
+  p.gcnt = h->ws.split_cnt;
+  p.max_entries = h->ws.split_entries;
   p.err = h->ws.err;
+  // mode 0 both passes, 1 pass 1 only (row statistics), 2 pass 2 only
+  auto kernel = mode == 1 ? attn_tc_kernel<1> : mode == 2 ? attn_tc_kernel<2> : attn_tc_kernel<0>;
   const size_t smem = attn_tc_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  e = launch_pdl_if(h->pdl, attn_tc_kernel, dim3(h->num_sms), dim3(THREADS), smem, st, h->tm_q, tm_k, tm_v, p);
+  e = launch_pdl_if(h->pdl, kernel, dim3(h->num_sms), dim3(THREADS), smem, st, h->tm_q, tm_k, tm_v, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

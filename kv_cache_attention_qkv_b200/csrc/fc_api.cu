@@ -150,8 +150,9 @@ static fc_status validate_config(const fc_config* c) {
 
 static void free_workspace(fc_handle* h) {
   fc::Workspace& w = h->ws;
-  void* ptrs[] = {w.q_buf, w.row_dst,  w.imp_acc,  w.items,   w.sched,
-                  w.err,   w.rope_cos, w.rope_sin, w.items_fb};
+  void* ptrs[] = {w.q_buf,    w.row_dst,  w.imp_acc,     w.items,   w.sched,
+                  w.err,      w.rope_cos, w.rope_sin,    w.items_fb, w.split_stats,
+                  w.split_o,  w.split_cnt};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   w = fc::Workspace{};
@@ -189,6 +190,11 @@ fc_status fc_create(const fc_config* cfg, const void* w_qkv, fc_handle** out) {
 
   const int qtile = h->tc_attn ? fc::kTcQTile : fc::kSimtQTile;
   h->ws.max_items = H * (cfg->max_total_q / qtile + cfg->max_batch + 1);
+  // a split small batch has at most one entry per SM
+  if (h->tc_attn) {
+    h->ws.split_entries = nsm;
+    if (h->ws.max_items < nsm) h->ws.max_items = nsm;
+  }
 
   fc::Workspace& w = h->ws;
   size_t es = elem_size(cfg->dtype);
@@ -202,7 +208,12 @@ fc_status fc_create(const fc_config* cfg, const void* w_qkv, fc_handle** out) {
             cudaMalloc(&w.rope_cos, (size_t)cfg->max_pos * half * sizeof(float)) == cudaSuccess &&
             cudaMalloc(&w.rope_sin, (size_t)cfg->max_pos * half * sizeof(float)) == cudaSuccess;
   if (ok && h->tc_attn)
-    ok = cudaMalloc(&w.items_fb, (size_t)w.max_items * sizeof(fc::WorkItem)) == cudaSuccess;
+    ok = cudaMalloc(&w.items_fb, (size_t)w.max_items * sizeof(fc::WorkItem)) == cudaSuccess &&
+         cudaMalloc(&w.split_stats, (size_t)w.split_entries * 256 * sizeof(float)) == cudaSuccess &&
+         cudaMalloc(&w.split_o, (size_t)w.split_entries * 128 * 128 * sizeof(float)) ==
+             cudaSuccess &&
+         cudaMalloc(&w.split_cnt, (size_t)w.split_entries * sizeof(int32_t)) == cudaSuccess &&
+         cudaMemset(w.split_cnt, 0, (size_t)w.split_entries * sizeof(int32_t)) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     free_workspace(h);
@@ -312,14 +323,25 @@ fc_status fc::step_impl(fc_handle* h, const CUtensorMap* tm_w, void* stream, int
   }
   StepShape s{batch, total_q, total_k, c.hidden, c.n_heads, c.head_dim, c.max_pos, c.max_seqlen_q};
   const bool want_imp = importance != nullptr;
+  // A small batch (at most one 128-row item per SM even if every sequence
+  // ends in a partial query tile) with long caches (2048 rows or more on
+  // average) splits its items' caches over the SMs and runs the two attention
+  // passes as two launches.  Each launch costs several microseconds of fixed
+  // latency, so shorter caches stay on the single launch.
+  const bool split_attn =
+      h->tc_attn && h->attn_split != 1 &&
+      (long long)c.n_heads * ((total_q + fc::kTcQTile - 1) / fc::kTcQTile + batch - 1) <=
+          h->ws.split_entries &&
+      (h->attn_split == 2 || (long long)total_k >= 2048LL * batch);
   cudaError_t e;
   {
     ProfScope ps(h, st, 0);
-    // tensor-core path: with importance every item goes to the two-pass
-    // kernel (long_tiles 0), without it to the one-pass kernel
+    // tensor-core path: with importance (or split) every item goes to the
+    // two-pass kernel (long_tiles 0), without it to the one-pass kernel
     e = fc::launch_prep(h, st, s, q_pos, cu_seqlens_q, cu_seqlens_k,
                         h->tc_attn ? fc::kTcQTile : fc::kSimtQTile,
-                        (h->tc_attn && want_imp) ? 0 : 0x7fffffff);
+                        (h->tc_attn && (want_imp || split_attn)) ? 0 : 0x7fffffff,
+                        split_attn ? h->ws.split_entries : 0, h->attn_split == 2 ? 1 : 4);
   }
   if (e != cudaSuccess) return cuda_fail(h, 0, e);
   h->last_launches++;
@@ -345,10 +367,21 @@ fc_status fc::step_impl(fc_handle* h, const CUtensorMap* tm_w, void* stream, int
     if (!fc::encode_kv_3d(&tm_k, k_cache, total_k, c.n_heads) ||
         !fc::encode_kv_3d(&tm_v, v_cache, total_k, c.n_heads))
       return cuda_fail(h, -1, cudaErrorInvalidValue);
-    if (want_imp) {
+    if (split_attn) {
+      // pass 1 of every entry (row statistics), then pass 2 and the combine
+      {
+        ProfScope ps(h, st, 8);
+        e = fc::launch_attn_tc(h, st, s, tm_k, tm_v, cu_seqlens_q, cu_seqlens_k, out, want_imp, 1);
+      }
+      if (e != cudaSuccess) return cuda_fail(h, 8, e);
+      h->last_launches++;
+      ProfScope ps(h, st, 2);
+      e = fc::launch_attn_tc(h, st, s, tm_k, tm_v, cu_seqlens_q, cu_seqlens_k, out, want_imp, 2);
+      if (e != cudaSuccess) return cuda_fail(h, 2, e);
+    } else if (want_imp) {
       // the importance needs every row's final normaliser: two scans of K
       ProfScope ps(h, st, 2);
-      e = fc::launch_attn_tc(h, st, s, tm_k, tm_v, cu_seqlens_q, cu_seqlens_k, out, true);
+      e = fc::launch_attn_tc(h, st, s, tm_k, tm_v, cu_seqlens_q, cu_seqlens_k, out, true, 0);
       if (e != cudaSuccess) return cuda_fail(h, 2, e);
     } else {
       {
@@ -359,7 +392,7 @@ fc_status fc::step_impl(fc_handle* h, const CUtensorMap* tm_w, void* stream, int
       h->last_launches++;
       // the items the one-pass kernel handed over (usually none)
       ProfScope ps(h, st, 2);
-      e = fc::launch_attn_tc(h, st, s, tm_k, tm_v, cu_seqlens_q, cu_seqlens_k, out, false);
+      e = fc::launch_attn_tc(h, st, s, tm_k, tm_v, cu_seqlens_q, cu_seqlens_k, out, false, 0);
       if (e != cudaSuccess) return cuda_fail(h, 2, e);
     }
   } else {
@@ -463,13 +496,18 @@ fc_status fc_set_option(fc_handle* h, int option, int value) {
     h->qkv_split = value;
     return FC_OK;
   }
+  if (option == FC_OPT_ATTN_SPLIT) {
+    if (value < 0 || value > 2) return FC_ERR_INVALID_ARG;
+    h->attn_split = value;
+    return FC_OK;
+  }
   return FC_ERR_INVALID_ARG;
 }
 
 const char* fc_last_cuda_error(const fc_handle* h) {
   static const char* const kSlot[] = {"prep", "qkv_rope_scatter", "attention",
                                       "importance_finalize", "topk", "attention_one_pass",
-                                      "h2d_copy", "d2h_copy"};
+                                      "h2d_copy", "d2h_copy", "attention_split_pass1"};
   static thread_local char buf[256];
   if (!h || h->last_cuda_err == cudaSuccess) return "no CUDA error recorded";
   snprintf(buf, sizeof(buf), "%s: %s (%s)",

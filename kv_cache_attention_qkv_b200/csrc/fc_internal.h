@@ -80,6 +80,11 @@ struct Workspace {
   float* rope_cos = nullptr;              // [max_pos, d/2]
   float* rope_sin = nullptr;              // [max_pos, d/2]
   int max_items = 0;
+  // small batches, items split over several CTAs (tensor-core attention):
+  float* split_stats = nullptr;           // [split_entries][m, l][128]
+  float* split_o = nullptr;               // [split_entries][128][128] fp32 parts of O
+  int32_t* split_cnt = nullptr;           // [split_entries] finished entries per item
+  int split_entries = 0;
 };
 
 // Shapes of one step, as the kernels see them.
@@ -129,6 +134,7 @@ struct fc_handle {
   // pair kernel, 2 the split-K cluster kernel (fc_set_option)
   int qkv_kernel = 0;
   int qkv_split = 0;  // split-K cluster size: 0 chosen by shape, else forced
+  int attn_split = 0;  // small-batch attention split: 0 by shape, 1 never
   // resident clusters of the split-K projection kernel per cluster size 2..8
   int splitk_clusters[9] = {};
   // the last CUDA call of fc_step that failed: its error and the profile slot
@@ -193,7 +199,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // ---- launchers (each returns the CUDA error of its launch) -----------------
 cudaError_t launch_prep(const fc_handle* h, cudaStream_t st, const StepShape& s,
                         const int32_t* q_pos, const int32_t* cu_q, const int32_t* cu_k,
-                        int qtile, int long_tiles);
+                        int qtile, int long_tiles, int split_sms, int split_min_tiles);
 cudaError_t launch_qkv_simt(const fc_handle* h, cudaStream_t st, const StepShape& s,
                             const void* x, const int32_t* q_pos, void* k_cache, void* v_cache);
 cudaError_t launch_attn_simt(const fc_handle* h, cudaStream_t st, const StepShape& s,
@@ -227,7 +233,7 @@ fc_status step_impl(fc_handle* h, const CUtensorMap* tm_w, void* stream, int bat
 cudaError_t launch_attn_tc(const fc_handle* h, cudaStream_t st, const StepShape& s,
                            const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                            const int32_t* cu_q, const int32_t* cu_k, void* out,
-                           bool want_importance);
+                           bool want_importance, int mode);
 cudaError_t launch_attn_onepass(const fc_handle* h, cudaStream_t st, const CUtensorMap& tm_k,
                                 const CUtensorMap& tm_v, const int32_t* cu_q, const int32_t* cu_k,
                                 void* out);

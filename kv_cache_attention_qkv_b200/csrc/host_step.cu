@@ -13,6 +13,10 @@ namespace {
 
 size_t align16(size_t n) { return (n + 15) & ~(size_t)15; }
 
+// input + output bytes of a call from which its kernels are fenced by timed
+// events (see fc_step_host)
+constexpr size_t kFenceCopyBytes = 16u << 20;
+
 // int32 offsets of the small arrays inside one staging block
 struct SmallLayout {
   size_t q_pos, cu_q, cu_k, lo, hi, kps, total;  // in int32 elements
@@ -143,15 +147,21 @@ fc_status fc_step_host(fc_handle* h, void* stream, int batch, const void* x, con
   if (e == cudaSuccess && reuse) e = cudaStreamWaitEvent(cs, p.d2h_done[s], 0);
   if (e != cudaSuccess) return FC_ERR_CUDA;
   // The kernels run here beside the input copy of the next call and the
-  // output copy of the previous one.  Launched back to back they stretched
-  // the input copy (batch 32 x 128 rows, 33.5 MB: 1.05 ms at 32 GB/s instead
-  // of 0.75 ms at 44 GB/s) and the step to 1.0-1.05 ms; with a timed event
-  // recorded on each side of every kernel (which also ends programmatic
-  // overlap between them, so the kernels are launched plainly) the step takes
-  // 0.77-0.80 ms, near the two copies' concurrent rate.  Timing-disabled
-  // events, or timed events around a single kernel, did not help.
-  h->pdl = false;
-  p.fencing = true;
+  // output copy of the previous one.  With large copies (batch 32 x 128 rows:
+  // 33.5 MB each way), kernels launched back to back stretched the input copy
+  // (1.05 ms at 32 GB/s instead of 0.75 ms at 44 GB/s) and the step to
+  // 1.0-1.05 ms; with a timed event recorded on each side of every kernel
+  // (which also ends programmatic overlap between them, so the kernels are
+  // launched plainly) the step takes 0.77-0.80 ms, near the two copies'
+  // concurrent rate.  Timing-disabled events, or timed events around a single
+  // kernel, did not help.  Small steps are latency-bound instead (batch 1:
+  // 1 MB each way), and there the events cost more than they save, so they
+  // keep the device path's launches.
+  const bool big_copies = x_bytes + out_bytes >= kFenceCopyBytes;
+  if (big_copies) {
+    h->pdl = false;
+    p.fencing = true;
+  }
   st = fc_step(h, stream, batch, p.x[s], sm + L.q_pos, sm + L.cu_q, sm + L.cu_k, total_q, total_k,
                k_cache, v_cache, p.out[s], p.importance, 0);
   const int step_launches = h->last_launches;

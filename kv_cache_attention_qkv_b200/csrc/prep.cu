@@ -30,6 +30,14 @@ __device__ __forceinline__ bool seq_ok(const int32_t* cu_q, const int32_t* cu_k,
 // sequences whose cache spans more than long_tiles 128-key tiles come first
 // (the list is ordered by cache length); sched[2] counts them: the two-pass
 // attention kernel takes those, the one-pass kernel the rest.
+//
+// With split_sms > 0 (a small batch), every item is cut into
+// ns = max(1, min(split_sms / items, 8, its key tiles / split_min_tiles))
+// entries over nearly equal runs of key tiles, so that the entries fill up to
+// split_sms CTAs and each keeps at least split_min_tiles tiles.  An entry
+// records its key tiles [j0, j1) in pad[0] (j0 | j1 << 16) and its item's
+// first entry and entry count in pad[1] (first | ns << 28); without a split,
+// ns = 1 and [j0, j1) covers the whole cache.
 __global__ void __launch_bounds__(512) prep_kernel(StepShape s, const int32_t* __restrict__ q_pos,
                                                    const int32_t* __restrict__ cu_q,
                                                    const int32_t* __restrict__ cu_k,
@@ -37,7 +45,8 @@ __global__ void __launch_bounds__(512) prep_kernel(StepShape s, const int32_t* _
                                                    WorkItem* __restrict__ items, int max_items,
                                                    int32_t* __restrict__ sched,
                                                    int32_t* __restrict__ err, int qtile,
-                                                   int long_tiles) {
+                                                   int long_tiles, int split_sms,
+                                                   int split_min_tiles) {
   extern __shared__ uint32_t smem[];
   const int b = blockIdx.x;
   const int tid = threadIdx.x, nt = blockDim.x;
@@ -127,6 +136,7 @@ __global__ void __launch_bounds__(512) prep_kernel(StepShape s, const int32_t* _
   }
   int* sseq = cnt + n2;   // [n2] sequence of each sorted slot
   int* snq = sseq + n2;   // [n2] query tiles of each sorted slot
+  int* sns = snq + n2;    // [n2] entries per item of each sorted slot
   for (int i = tid; i < n2; i += nt) {
     int c = 0, bq = 0, nqt = 0;
     if (i < s.B && (key[i] >> 63)) {
@@ -140,7 +150,24 @@ __global__ void __launch_bounds__(512) prep_kernel(StepShape s, const int32_t* _
     snq[i] = nqt;
   }
   __syncthreads();
-  if (tid < 32) {  // exclusive scan of cnt[0 .. B) by one warp
+  if (tid < 32) {
+    // entries per item: split the items of a small batch over the SMs
+    int groups = 0;
+    for (int i = tid; i < s.B; i += 32) groups += cnt[i];
+    for (int o = 16; o > 0; o >>= 1) groups += __shfl_xor_sync(0xffffffffu, groups, o);
+    int target = 1;
+    if (split_sms > 0 && groups > 0) target = max(1, min(8, split_sms / groups));
+    for (int i = tid; i < s.B; i += 32) {
+      int ns = 1;
+      if (cnt[i] > 0) {
+        const int L = (int)((key[i] >> 32) & 0x7FFFFFFFull);
+        ns = max(1, min(target, (L + 127) / 128 / max(split_min_tiles, 1)));
+      }
+      sns[i] = ns;
+      cnt[i] *= ns;
+    }
+    __syncwarp();
+    // exclusive scan of cnt[0 .. B) by one warp
     int carry = 0;
     for (int base = 0; base < s.B; base += 32) {
       const int i = base + tid;
@@ -173,14 +200,20 @@ __global__ void __launch_bounds__(512) prep_kernel(StepShape s, const int32_t* _
   __syncthreads();
   for (int i = 0; i < s.B; ++i) {
     if (!(key[i] >> 63)) break;
-    const int bq = sseq[i], nqt = snq[i];
-    const int c = s.H * nqt;
+    const int bq = sseq[i], nqt = snq[i], ns = sns[i];
+    const int c = s.H * nqt * ns;
     const int off = cnt[i];
     const int q0 = cu_q[bq], n = cu_q[bq + 1] - q0, k0 = cu_k[bq], L = cu_k[bq + 1] - k0;
+    const int ntiles = (L + 127) / 128;
     for (int t = tid; t < c; t += nt) {
-      const int hh = t / nqt, qt = t - hh * nqt;
+      const int g = t / ns, sp = t - g * ns;
+      const int hh = g / nqt, qt = g - hh * nqt;
+      const int j0 = sp * ntiles / ns, j1 = (sp + 1) * ntiles / ns;
+      const int first = off + g * ns;
       if (off + t < max_items)
-        items[off + t] = WorkItem{bq, (qt << 8) | hh, q0, min(qtile, n - qt * qtile), k0, L, {0, 0}};
+        items[off + t] = WorkItem{bq, (qt << 8) | hh, q0, min(qtile, n - qt * qtile), k0, L,
+                                  {(int)((unsigned)j0 | ((unsigned)j1 << 16)),
+                                   (int)((unsigned)first | ((unsigned)ns << 28))}};
     }
   }
 }
@@ -191,13 +224,13 @@ size_t prep_smem_bytes(int max_pos, int max_batch) {
   size_t bitmap = 2u * (size_t)((max_pos + 31) / 32) * sizeof(uint32_t);
   int n2 = 1;
   while (n2 < max_batch) n2 <<= 1;
-  size_t sortb = (size_t)n2 * (sizeof(unsigned long long) + 3 * sizeof(int));
+  size_t sortb = (size_t)n2 * (sizeof(unsigned long long) + 4 * sizeof(int));
   return bitmap > sortb ? bitmap : sortb;
 }
 
 cudaError_t launch_prep(const fc_handle* h, cudaStream_t st, const StepShape& s,
                         const int32_t* q_pos, const int32_t* cu_q, const int32_t* cu_k,
-                        int qtile, int long_tiles) {
+                        int qtile, int long_tiles, int split_sms, int split_min_tiles) {
   size_t smem = prep_smem_bytes(h->cfg.max_pos, h->cfg.max_batch);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -206,7 +239,7 @@ cudaError_t launch_prep(const fc_handle* h, cudaStream_t st, const StepShape& s,
   }
   prep_kernel<<<s.B + 1, 512, smem, st>>>(s, q_pos, cu_q, cu_k, h->ws.row_dst, h->ws.items,
                                            h->ws.max_items, h->ws.sched, h->ws.err, qtile,
-                                           long_tiles);
+                                           long_tiles, split_sms, split_min_tiles);
   return cudaGetLastError();
 }
 

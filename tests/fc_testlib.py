@@ -56,10 +56,16 @@ def make_layer(inp: workloads.StepInputs, w: torch.Tensor, **over):
     return FlashCache(w, **kw)
 
 
-def run_gpu(inp: workloads.StepInputs, layer=None, dev=None, want_importance=True):
-    """One fc_step + fc_topk_tracked; returns numpy results and the device state."""
+def run_gpu(inp: workloads.StepInputs, layer=None, dev=None, want_importance=True,
+            attn_split=True):
+    """One fc_step + fc_topk_tracked; returns numpy results and the device state.
+    ``attn_split``: True (the default rule), False (never split a small batch's
+    attention) or "always" (split a small batch whatever its cache length)."""
     dev = dev or upload(inp)
-    layer = layer or make_layer(inp, dev["w"])
+    if layer is None:
+        layer = make_layer(inp, dev["w"])
+        if attn_split is not True:
+            layer.set_attn_split(attn_split)
     T, H, d = inp.total_q, inp.n_heads, inp.head_dim
     out = torch.full((T, H, d), float("nan"), device=dev["x"].device, dtype=dev["x"].dtype)
     imp = torch.full((inp.total_k,), float("nan"), device=dev["x"].device) if want_importance else None
@@ -77,6 +83,27 @@ def run_gpu(inp: workloads.StepInputs, layer=None, dev=None, want_importance=Tru
     res["err"] = layer.get_error()
     res["out"] = out.float().cpu().numpy().astype(np.float64)
     return res
+
+
+def split_entries(inp: workloads.StepInputs, num_sms: int, forced=False) -> int:
+    """Work entries of a small batch whose items are split over the SMs: every
+    (sequence, head, 128-row tile) item becomes max(1, min(target, its 128-key
+    tiles // m)) entries, target = min(8, SMs // items), m = 4 (1 when the
+    split is forced)."""
+    n = np.diff(inp.cu_seqlens_q)
+    L = np.diff(inp.cu_seqlens_k)
+    live = (n > 0) & (L > 0)
+    items = inp.n_heads * ((n + 127) // 128) * live
+    target = max(1, min(8, num_sms // max(int(items.sum()), 1)))
+    ns = np.maximum(1, np.minimum(target, (L + 127) // 128 // (1 if forced else 4)))
+    return int((items * ns).sum())
+
+
+def splits_attention(inp: workloads.StepInputs, num_sms: int, forced=False) -> bool:
+    """Whether fc_step takes the small-batch split path for these shapes (by
+    default: small batch and caches of 2048 rows or more on average)."""
+    small = inp.n_heads * ((inp.total_q + 127) // 128 + inp.batch - 1) <= num_sms
+    return small and (forced or inp.total_k >= 2048 * inp.batch)
 
 
 def run_oracle(inp: workloads.StepInputs, seqs: Optional[Iterable[int]] = None):

@@ -153,3 +153,11 @@ def test_step_result_line_follows_the_contract():
     ni = r2["no_importance"]
     assert ni["ms_per_step"] == pytest.approx(0.3)
     assert ni["attention_one_pass"]["achieved"] == pytest.approx(wk["attn_bytes"] / 0.04e-3 / 1e9)
+    # a split small batch: its attention is the sum of its two launches
+    pk3 = dict(per_kernel)
+    pk3["attention_split_pass1"] = (0.5, 10)
+    r3 = bench._step_result(args, inp, 2, total_ms=5.0, burst_ms=4.0, per_kernel=pk3,
+                            launches=50, err=0, e2e_ms=8.0, h2d=1000, d2h=2000, clocks=clocks,
+                            num_sms=148)
+    att3 = r3["kernel_rooflines"]["attention"]
+    assert att3["achieved"] == pytest.approx(wk["attn_bytes"] / ((2.0 + 0.5) / 10 * 1e-3) / 1e9)

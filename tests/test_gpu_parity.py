@@ -86,17 +86,69 @@ def test_full_size_sampled_parity(name, seqs):
 
 
 def test_attention_work_split():
-    """A step with importance gives every item to the two-pass kernel (the column
-    sums need each row's final normaliser); a step without importance gives
-    them to the one-pass kernel, whose ordinary scores never leave its
-    exponent band."""
+    """Unsplit, a step with importance gives every item to the two-pass kernel
+    (the column sums need each row's final normaliser) and a step without
+    importance gives them to the one-pass kernel, whose ordinary scores never
+    leave its exponent band.  Split (forced: its caches are short), every item
+    becomes entries over runs of key tiles, all in the two-pass kernel."""
     inp = workloads.generate("small_longcache")
     n = np.diff(inp.cu_seqlens_q)
     want = inp.n_heads * int(((n + 127) // 128).sum())
-    gpu = tl.run_gpu(inp)
+    gpu = tl.run_gpu(inp, attn_split=False)
     assert gpu["layer"].last_step_work() == (want, want, 0)
-    g = tl.run_gpu(inp, want_importance=False)
+    g = tl.run_gpu(inp, want_importance=False, attn_split=False)
     assert g["layer"].last_step_work() == (want, 0, 0)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert not tl.splits_attention(inp, sms) and tl.splits_attention(inp, sms, forced=True)
+    entries = tl.split_entries(inp, sms, forced=True)
+    assert entries > want
+    for imp in (True, False):
+        g = tl.run_gpu(inp, want_importance=imp, attn_split="always")
+        assert g["layer"].last_step_work() == (entries, entries, 0)
+
+
+@pytest.mark.parametrize("name", ["small_varlen", "small_longcache", "layer_b1"])
+def test_split_attention_agrees_with_unsplit(name):
+    """The small-batch split (forced here: these caches are short; two launches,
+    parts of O combined by the item's last entry in entry order) against the
+    oracle, with and without importance, and run to run bit-identical; the
+    unsplit kernels agree within the bar."""
+    inp = workloads.generate(name)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert tl.splits_attention(inp, sms, forced=True)
+    ref = tl.run_oracle(inp)
+    for imp in (True, False):
+        a = tl.run_gpu(inp, want_importance=imp, attn_split="always")
+        b = tl.run_gpu(inp, want_importance=imp, attn_split="always")
+        u = tl.run_gpu(inp, want_importance=imp, attn_split=False)
+        for g in (a, u):
+            assert g["err"] == 0
+            tl.compare_step(inp, g, ref, range(inp.batch))
+        assert np.array_equal(a["out"], b["out"])
+        tl.assert_close(a["out"], u["out"], tl.TOL[inp.dtype], "split vs unsplit")
+        if imp:
+            assert np.array_equal(a["importance"], b["importance"])
+            tl.assert_close(a["importance"], ref["importance"], tl.TOL[inp.dtype], "importance")
+            np.testing.assert_array_equal(a["tracked"], b["tracked"])
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,seqs", [("sweep_b1_m128_L8192", [0]), ("sweep_b2_m128_L8192", [0, 1]),
+                                       ("sweep_b1_m128_L1536", [0]), ("sweep_b2_m256_L8192", [0, 1])])
+def test_split_attention_full_size(name, seqs):
+    """Small batches at full size, in the launch configuration the bench uses
+    (split for the long caches, not for L = 1536 nor for beta = 256 at B = 2),
+    against the oracle."""
+    inp = workloads.generate(name)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    gpu = tl.run_gpu(inp)
+    assert gpu["err"] == 0
+    if tl.splits_attention(inp, sms):
+        e = tl.split_entries(inp, sms)
+        assert gpu["layer"].last_step_work() == (e, e, 0)
+    ref = tl.run_oracle(inp, seqs=seqs)
+    tl.compare_step(inp, gpu, ref, seqs)
+    tl.assert_unwritten_rows_unchanged(inp, gpu)
 
 
 @pytest.mark.parametrize("name,seqs", [("small_varlen", None), ("small_longcache", None),
@@ -104,7 +156,7 @@ def test_attention_work_split():
 def test_one_pass_attention_without_importance(name, seqs):
     """The one-pass kernel (steps without importance) against the oracle."""
     inp = workloads.generate(name)
-    gpu = tl.run_gpu(inp, want_importance=False)
+    gpu = tl.run_gpu(inp, want_importance=False, attn_split=False)
     assert gpu["err"] == 0
     ref = tl.run_oracle(inp, seqs=seqs)
     tl.compare_step(inp, gpu, ref, seqs if seqs is not None else range(inp.batch))
@@ -163,16 +215,21 @@ def test_scores_out_of_the_one_pass_band_are_handed_over(seq):
     oracle."""
     inp = workloads.generate("small_varlen")
     _plant_far_key(inp, seq, 64, seed=seq)
-    gpu = tl.run_gpu(inp, want_importance=False)
+    gpu = tl.run_gpu(inp, want_importance=False, attn_split=False)
     assert gpu["err"] == 0
     items, two_pass, handed = gpu["layer"].last_step_work()
     assert two_pass == 0 and handed == inp.n_heads  # every head of that sequence
     ref = tl.run_oracle(inp)
     tl.compare_step(inp, gpu, ref, range(inp.batch))
     # with importance the same step runs in the two-pass kernel from the start
-    g2 = tl.run_gpu(inp)
+    g2 = tl.run_gpu(inp, attn_split=False)
     assert g2["layer"].last_step_work()[2] == 0
     tl.compare_step(inp, g2, ref, range(inp.batch))
+    # split over the SMs (two launches), with and without importance
+    for imp in (True, False):
+        g3 = tl.run_gpu(inp, want_importance=imp, attn_split="always")
+        assert g3["err"] == 0
+        tl.compare_step(inp, g3, ref, range(inp.batch))
 
 
 def test_topk_kernel_is_exact_on_gpu_importance():
