@@ -12,6 +12,14 @@
 // larger scores are kept, equal ones in position order until k are kept, and
 // the kept set is sorted by (score desc, position asc).  The result does not
 // depend on thread timing.
+//
+// Small selections (k <= 64 from at most 2048 candidates, the usual case) take
+// a path with five block barriers instead of about forty: each of the 16 warps
+// sorts up to 128 candidates in registers (bitonic network over composite
+// keys score << 32 | ~position, so ties go to the lower position), keeps its
+// 64 largest, and the warps' lists are merged pairwise in four rounds (the 64
+// largest of two sorted lists form a bitonic sequence, sorted by one
+// half-cleaner network).
 #include "fc_internal.h"
 #include "ptx.cuh"
 
@@ -34,6 +42,45 @@ __global__ void importance_finalize(int S, unsigned long long* __restrict__ acc,
 __device__ __forceinline__ uint32_t fkey(float f) {
   uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
+  return ((unsigned long long)hi << 32) | lo;
+}
+
+// Sort the warp's 32 * R keys descending; element e = 32 * r + lane is v[r].
+template <int R>
+__device__ __forceinline__ void warp_bitonic_desc(unsigned long long (&v)[R], int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32 * R; size <<= 1) {
+#pragma unroll
+    for (int j = size >> 1; j > 0; j >>= 1) {
+      if (j >= 32) {
+        const int rj = j >> 5;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          if (r & rj) continue;
+          const bool desc = ((32 * r + lane) & size) == 0;
+          const unsigned long long a = v[r], b = v[r | rj];
+          const bool sw = desc ? (a < b) : (a > b);
+          v[r] = sw ? b : a;
+          v[r | rj] = sw ? a : b;
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const int e = 32 * r + lane;
+          const bool desc = (e & size) == 0;
+          const unsigned long long o = shfl_xor_u64(v[r], j);
+          const bool lower = (lane & j) == 0;  // e is the lower index of the pair
+          const bool keep_max = lower == desc;
+          v[r] = keep_max ? (v[r] > o ? v[r] : o) : (v[r] < o ? v[r] : o);
+        }
+      }
+    }
+  }
 }
 
 constexpr int TK_THREADS = 512;
@@ -76,6 +123,58 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(
     __syncthreads();
   }
   auto key_of = [&](int i) { return staged ? skey[i] : fkey(sc[i]); };
+
+  if (want > 0 && want <= 64 && n <= (TK_THREADS / 32) * 128) {
+    // ---- small selection: per-warp register sort, then a pairwise merge
+    const int per = (n + TK_THREADS / 32 - 1) / (TK_THREADS / 32);  // candidates per warp, <= 128
+    const int c0 = warp * per;
+    unsigned long long v[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int idx = 32 * r + lane, i = c0 + idx;
+      v[r] = (idx < per && i < n)
+                 ? ((unsigned long long)skey[i] << 32) | (0xFFFFFFFFu - (uint32_t)(lo + i))
+                 : 0ull;  // below every candidate's composite key
+    }
+    warp_bitonic_desc<4>(v, lane);
+    unsigned long long* buf[2] = {sel, reinterpret_cast<unsigned long long*>(skey)};
+    buf[0][warp * 64 + lane] = v[0];
+    buf[0][warp * 64 + 32 + lane] = v[1];
+    __syncthreads();  // every warp has also finished reading skey
+    int cur = 0;
+    for (int lists = TK_THREADS / 32; lists > 1; lists >>= 1) {
+      if (warp < lists / 2) {
+        const unsigned long long* A = buf[cur] + (2 * warp) * 64;
+        const unsigned long long* B = A + 64;
+        unsigned long long m[2];
+        m[0] = A[lane] > B[63 - lane] ? A[lane] : B[63 - lane];
+        m[1] = A[32 + lane] > B[31 - lane] ? A[32 + lane] : B[31 - lane];
+        // m is bitonic: half-cleaner stages 32, 16, ..., 1 sort it descending
+        {
+          const unsigned long long a = m[0], b = m[1];
+          m[0] = a > b ? a : b;
+          m[1] = a > b ? b : a;
+        }
+#pragma unroll
+        for (int j = 16; j > 0; j >>= 1) {
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const unsigned long long o = shfl_xor_u64(m[r], j);
+            const bool lower = (lane & j) == 0;
+            m[r] = lower ? (m[r] > o ? m[r] : o) : (m[r] < o ? m[r] : o);
+          }
+        }
+        unsigned long long* D = buf[cur ^ 1] + warp * 64;
+        D[lane] = m[0];
+        D[32 + lane] = m[1];
+      }
+      __syncthreads();
+      cur ^= 1;
+    }
+    for (int i = tid; i < k; i += TK_THREADS)
+      row[i] = i < want ? (int32_t)(0xFFFFFFFFu - (uint32_t)(buf[cur][i] & 0xFFFFFFFFull)) : -1;
+    return;
+  }
 
   // ---- radix select of the want-th largest key
   uint32_t prefix = 0u, mask = 0u;
