@@ -914,11 +914,15 @@ def run_e2e_timeline(args):
 
 # Sweep axes (the pages' measured axes, throughput side): batch size at the
 # headline query and cache, query size beta_m at batch 32, cache length at
-# batch 32 and beta_m 128.
+# batch 32 and beta_m 128, and cache length at batch 1-4.
 SWEEPS = {
     "batch": [f"sweep_b{b}_m128_L1536" for b in (1, 2, 4, 8, 16, 32, 64)],
     "beta": [f"sweep_b32_m{m}_L1536" for m in (64, 128, 192, 256)],
     "cache": [f"sweep_b32_m128_L{L}" for L in (768, 1536, 3072, 4096, 8192)],
+    # small batches with long caches: the attention split over the SMs (B = 1, 2 from 2048 rows
+    # on average; B = 4 has too many items to split)
+    "small_batch_long_cache": [f"sweep_b{b}_m128_L{L}" for b, L in
+                               ((1, 1536), (1, 2048), (1, 4096), (1, 8192), (2, 8192), (4, 8192))],
 }
 
 
