@@ -919,7 +919,7 @@ SWEEPS = {
     "batch": [f"sweep_b{b}_m128_L1536" for b in (1, 2, 4, 8, 16, 32, 64)],
     "beta": [f"sweep_b32_m{m}_L1536" for m in (64, 128, 192, 256)],
     "cache": [f"sweep_b32_m128_L{L}" for L in (768, 1536, 3072, 4096, 8192)],
-    # small batches with long caches: the attention split over the SMs (B = 1, 2 from 2048 rows
+    # small batches with long caches: the attention split over the SMs (B = 1, 2 from 1280 rows
     # on average; B = 4 has too many items to split)
     "small_batch_long_cache": [f"sweep_b{b}_m128_L{L}" for b, L in
                                ((1, 1536), (1, 2048), (1, 4096), (1, 8192), (2, 8192), (4, 8192))],
@@ -952,7 +952,7 @@ def main():
                     help="cluster size of the split-K projection (default: the largest that fits at once)")
     ap.add_argument("--attn-split", choices=["auto", "never", "always"], default="auto",
                     help="small-batch attention split over the SMs (default: small batches "
-                         "with caches of 2048 rows or more)")
+                         "without importance or with caches of 1280 rows or more)")
     ap.add_argument("--sweep", choices=sorted(SWEEPS) + ["all"], default=None,
                     help="time every point of a sweep axis (one JSON line per point, no cpu_baseline)")
     args = ap.parse_args()

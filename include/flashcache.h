@@ -271,16 +271,16 @@ FC_API const char* fc_last_cuda_error(const fc_handle* h);
  *     with FC_ERR_INVALID_ARG.
  *   FC_OPT_ATTN_SPLIT: small-batch attention on the tensor-core path.  0
  *     (default): when H * (ceil(total_q / 128) + batch - 1) is at most the
- *     SM count and the caches hold 2048 rows or more on average
- *     (total_k >= 2048 * batch), every (sequence, head, 128-row query tile)
- *     item is split into max(1, min(SMs / items, 8, its 128-key tiles / 4))
- *     entries over runs of key tiles (at least four tiles each); a first launch stores each entry's row
+ *     SM count and either the step has no importance or the caches hold 1280
+ *     rows or more on average (total_k >= 1280 * batch), every (sequence,
+ *     head, 128-row query tile)
+ *     item is split into min(SMs / items, 8, its 128-key tiles) entries (at
+ *     least one) over runs of key tiles; a first launch stores each entry's row
  *     maxima and normalisers, a second combines them into the rows'
  *     log-sum-exp, computes P, P V and the column sums over its own keys, and
  *     the item's last entry adds the parts of O in entry order (so results do
  *     not depend on timing).  1: never split.  2: split whenever the batch is
- *     small enough, whatever the cache length, down to one tile per entry
- *     (for tests and measurement).
+ *     small enough, whatever the cache length (for tests and measurement).
  * FC_ERR_INVALID_ARG for an unknown option or value.
  */
 #define FC_OPT_QKV_KERNEL 1

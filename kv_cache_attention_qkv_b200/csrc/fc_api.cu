@@ -324,15 +324,19 @@ fc_status fc::step_impl(fc_handle* h, const CUtensorMap* tm_w, void* stream, int
   StepShape s{batch, total_q, total_k, c.hidden, c.n_heads, c.head_dim, c.max_pos, c.max_seqlen_q};
   const bool want_imp = importance != nullptr;
   // A small batch (at most one 128-row item per SM even if every sequence
-  // ends in a partial query tile) with long caches (2048 rows or more on
-  // average) splits its items' caches over the SMs and runs the two attention
-  // passes as two launches.  Each launch costs several microseconds of fixed
-  // latency, so shorter caches stay on the single launch.
+  // ends in a partial query tile) splits its items' caches over the SMs and
+  // runs the two attention passes as two launches when its caches hold 1280
+  // rows or more on average, or when the step has no importance (its unsplit
+  // path is two launches as well: the one-pass kernel and the hand-over
+  // kernel).  With importance and shorter caches the single two-pass launch
+  // is as fast or faster (each launch costs several microseconds of fixed
+  // latency; measured at B = 1: 768 rows 67.8 us unsplit vs 71.2 split, 1024
+  // rows 71.7 vs 72.7, 1536 rows 80.1 vs 75.5).
   const bool split_attn =
       h->tc_attn && h->attn_split != 1 &&
       (long long)c.n_heads * ((total_q + fc::kTcQTile - 1) / fc::kTcQTile + batch - 1) <=
           h->ws.split_entries &&
-      (h->attn_split == 2 || (long long)total_k >= 2048LL * batch);
+      (h->attn_split == 2 || !want_imp || (long long)total_k >= 1280LL * batch);
   cudaError_t e;
   {
     ProfScope ps(h, st, 0);
@@ -341,7 +345,7 @@ fc_status fc::step_impl(fc_handle* h, const CUtensorMap* tm_w, void* stream, int
     e = fc::launch_prep(h, st, s, q_pos, cu_seqlens_q, cu_seqlens_k,
                         h->tc_attn ? fc::kTcQTile : fc::kSimtQTile,
                         (h->tc_attn && (want_imp || split_attn)) ? 0 : 0x7fffffff,
-                        split_attn ? h->ws.split_entries : 0, h->attn_split == 2 ? 1 : 4);
+                        split_attn ? h->ws.split_entries : 0, 1);
   }
   if (e != cudaSuccess) return cuda_fail(h, 0, e);
   h->last_launches++;

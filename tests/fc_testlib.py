@@ -87,23 +87,24 @@ def run_gpu(inp: workloads.StepInputs, layer=None, dev=None, want_importance=Tru
 
 def split_entries(inp: workloads.StepInputs, num_sms: int, forced=False) -> int:
     """Work entries of a small batch whose items are split over the SMs: every
-    (sequence, head, 128-row tile) item becomes max(1, min(target, its 128-key
-    tiles // m)) entries, target = min(8, SMs // items), m = 4 (1 when the
-    split is forced)."""
+    (sequence, head, 128-row tile) item becomes min(target, its 128-key tiles)
+    entries, target = max(1, min(8, SMs // items))."""
     n = np.diff(inp.cu_seqlens_q)
     L = np.diff(inp.cu_seqlens_k)
     live = (n > 0) & (L > 0)
     items = inp.n_heads * ((n + 127) // 128) * live
     target = max(1, min(8, num_sms // max(int(items.sum()), 1)))
-    ns = np.maximum(1, np.minimum(target, (L + 127) // 128 // (1 if forced else 4)))
+    ns = np.maximum(1, np.minimum(target, (L + 127) // 128))
     return int((items * ns).sum())
 
 
-def splits_attention(inp: workloads.StepInputs, num_sms: int, forced=False) -> bool:
+def splits_attention(inp: workloads.StepInputs, num_sms: int, forced=False,
+                     importance=True) -> bool:
     """Whether fc_step takes the small-batch split path for these shapes (by
-    default: small batch and caches of 2048 rows or more on average)."""
+    default: a small batch without importance, or with caches of 1280 rows or
+    more on average)."""
     small = inp.n_heads * ((inp.total_q + 127) // 128 + inp.batch - 1) <= num_sms
-    return small and (forced or inp.total_k >= 2048 * inp.batch)
+    return small and (forced or not importance or inp.total_k >= 1280 * inp.batch)
 
 
 def run_oracle(inp: workloads.StepInputs, seqs: Optional[Iterable[int]] = None):
