@@ -100,7 +100,7 @@ struct AttnParams {
   unsigned long long* imp_acc;
   int want_imp;
   float* stats;  // [entry][m, l][128] row statistics of the entries (modes 1, 2)
-  float* opart;  // [entry][128][128] fp32 parts of O of split items (mode 2)
+  float* opart;  // [entry][128 columns][128 rows] fp32 parts of O of split items (mode 2)
   int32_t* gcnt; // [first entry of an item] entries of the item done (mode 2)
   int max_entries;
   int32_t* err;

@@ -82,7 +82,7 @@ struct Workspace {
   int max_items = 0;
   // small batches, items split over several CTAs (tensor-core attention):
   float* split_stats = nullptr;           // [split_entries][m, l][128]
-  float* split_o = nullptr;               // [split_entries][128][128] fp32 parts of O
+  float* split_o = nullptr;               // [split_entries][128 cols][128 rows] fp32 parts of O
   int32_t* split_cnt = nullptr;           // [split_entries] finished entries per item
   int split_entries = 0;
 };
