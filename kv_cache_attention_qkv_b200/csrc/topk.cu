@@ -13,13 +13,19 @@
 // the kept set is sorted by (score desc, position asc).  The result does not
 // depend on thread timing.
 //
-// Small selections (k <= 64 from at most 2048 candidates, the usual case) take
+// Small selections (k <= 64 from at most 8192 candidates, the usual case) take
 // a path with five block barriers instead of about forty: each of the 16 warps
-// sorts up to 128 candidates in registers (bitonic network over composite
-// keys score << 32 | ~position, so ties go to the lower position), keeps its
-// 64 largest, and the warps' lists are merged pairwise in four rounds (the 64
-// largest of two sorted lists form a bitonic sequence, sorted by one
-// half-cleaner network).
+// takes a run of up to 512 candidates in blocks of 128 and keeps the 64
+// largest seen so far, in registers, as composite keys score << 32 | ~position
+// (so ties go to the lower position).  The first block is sorted by a bitonic
+// network as wide as the run needs (32, 64 or 128 keys); of each later block
+// only the keys above the current 64th largest can enter, and when there are
+// at most 32 of them (the usual case once the running list has filled) they
+// are packed into one register and sorted alone.  The warps' lists are then
+// merged pairwise in four rounds.  Merging two sorted
+// lists of 64: their elementwise maxima against the other list reversed are
+// the 64 largest and form a bitonic sequence, sorted by one half-cleaner
+// network.
 #include "fc_internal.h"
 #include "ptx.cuh"
 
@@ -44,10 +50,35 @@ __device__ __forceinline__ uint32_t fkey(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+__device__ __forceinline__ unsigned long long shfl_idx_u64(unsigned long long v, int src) {
+  const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)v, src);
+  const uint32_t hi = __shfl_sync(0xffffffffu, (uint32_t)(v >> 32), src);
+  return ((unsigned long long)hi << 32) | lo;
+}
+
 __device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v, int m) {
   const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
   const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
   return ((unsigned long long)hi << 32) | lo;
+}
+
+// Sort the bitonic sequence of 64 keys m[0] (element lane), m[1] (element
+// 32 + lane) descending: half-cleaner stages 32, 16, ..., 1.
+__device__ __forceinline__ void warp_bitonic_merge64_desc(unsigned long long (&m)[2], int lane) {
+  {
+    const unsigned long long a = m[0], b = m[1];
+    m[0] = a > b ? a : b;
+    m[1] = a > b ? b : a;
+  }
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const unsigned long long o = shfl_xor_u64(m[r], j);
+      const bool lower = (lane & j) == 0;
+      m[r] = lower ? (m[r] > o ? m[r] : o) : (m[r] < o ? m[r] : o);
+    }
+  }
 }
 
 // Sort the warp's 32 * R keys descending; element e = 32 * r + lane is v[r].
@@ -119,28 +150,100 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(
   // up to TK_STAGE candidates are read from global memory once, as keys
   const bool staged = n <= TK_STAGE;
   if (staged && want > 0) {
-    for (int i = tid; i < n; i += TK_THREADS) skey[i] = fkey(sc[i]);
+    // eight independent loads in flight per thread (the stage is read once)
+    for (int base = 0; base < n; base += 8 * TK_THREADS) {
+      float f[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = base + u * TK_THREADS + tid;
+        f[u] = i < n ? __ldcg(sc + i) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = base + u * TK_THREADS + tid;
+        if (i < n) skey[i] = fkey(f[u]);
+      }
+    }
     __syncthreads();
   }
   auto key_of = [&](int i) { return staged ? skey[i] : fkey(sc[i]); };
 
-  if (want > 0 && want <= 64 && n <= (TK_THREADS / 32) * 128) {
-    // ---- small selection: per-warp register sort, then a pairwise merge
-    const int per = (n + TK_THREADS / 32 - 1) / (TK_THREADS / 32);  // candidates per warp, <= 128
+  if (staged && want > 0 && want <= 64) {
+    // ---- small selection: per-warp register sorts, then a pairwise merge
+    const int per = (n + TK_THREADS / 32 - 1) / (TK_THREADS / 32);  // candidates per warp, <= 512
     const int c0 = warp * per;
-    unsigned long long v[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int idx = 32 * r + lane, i = c0 + idx;
-      v[r] = (idx < per && i < n)
+    unsigned long long run[2] = {0ull, 0ull};  // the warp's 64 largest so far, descending
+    auto ckey = [&](int idx) -> unsigned long long {
+      const int i = c0 + idx;
+      return (idx < per && i < n)
                  ? ((unsigned long long)skey[i] << 32) | (0xFFFFFFFFu - (uint32_t)(lo + i))
                  : 0ull;  // below every candidate's composite key
+    };
+    // run = the 64 largest of run and the sorted list l0 (elements 0-31),
+    // l1 (32-63): element 63 - e of the list sits in lane 31 - lane of the
+    // other register
+    auto merge_into_run = [&](unsigned long long l0, unsigned long long l1) {
+      const unsigned long long r1 = shfl_xor_u64(l1, 31), r0 = shfl_xor_u64(l0, 31);
+      unsigned long long m[2];
+      m[0] = run[0] > r1 ? run[0] : r1;
+      m[1] = run[1] > r0 ? run[1] : r0;
+      warp_bitonic_merge64_desc(m, lane);
+      run[0] = m[0];
+      run[1] = m[1];
+    };
+    // first block: a network only as wide as the warp's run needs
+    if (per <= 32) {
+      unsigned long long v[1] = {ckey(lane)};
+      warp_bitonic_desc<1>(v, lane);
+      run[0] = v[0];
+    } else if (per <= 64) {
+      unsigned long long v[2] = {ckey(lane), ckey(32 + lane)};
+      warp_bitonic_desc<2>(v, lane);
+      run[0] = v[0];
+      run[1] = v[1];
+    } else {
+      unsigned long long v[4] = {ckey(lane), ckey(32 + lane), ckey(64 + lane), ckey(96 + lane)};
+      warp_bitonic_desc<4>(v, lane);
+      run[0] = v[0];
+      run[1] = v[1];
     }
-    warp_bitonic_desc<4>(v, lane);
+    // later blocks: only keys above the current 64th largest can enter; up to
+    // 32 of them are packed into one register (through this warp's slice of
+    // sel) and sorted alone
+    unsigned long long* pack = sel + warp * 64;
+    for (int b0 = 128; b0 < per; b0 += 128) {
+      const unsigned long long tau = shfl_idx_u64(run[1], 31);  // the 64th largest so far
+      unsigned long long v[4];
+      uint32_t bal[4];
+      int cnt = 0;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        v[r] = ckey(b0 + 32 * r + lane);
+        bal[r] = __ballot_sync(0xffffffffu, v[r] > tau);
+        cnt += __popc(bal[r]);
+      }
+      if (cnt == 0) continue;
+      if (cnt <= 32) {
+        int off = 0;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          if (v[r] > tau) pack[off + __popc(bal[r] & ((1u << lane) - 1u))] = v[r];
+          off += __popc(bal[r]);
+        }
+        __syncwarp();
+        unsigned long long x[1] = {lane < cnt ? pack[lane] : 0ull};
+        __syncwarp();
+        warp_bitonic_desc<1>(x, lane);
+        merge_into_run(x[0], 0ull);
+      } else {
+        warp_bitonic_desc<4>(v, lane);
+        merge_into_run(v[0], v[1]);
+      }
+    }
     unsigned long long* buf[2] = {sel, reinterpret_cast<unsigned long long*>(skey)};
-    buf[0][warp * 64 + lane] = v[0];
-    buf[0][warp * 64 + 32 + lane] = v[1];
-    __syncthreads();  // every warp has also finished reading skey
+    buf[0][warp * 64 + lane] = run[0];
+    buf[0][warp * 64 + 32 + lane] = run[1];
+    __syncthreads();  // every warp has also finished reading skey (buf[1])
     int cur = 0;
     for (int lists = TK_THREADS / 32; lists > 1; lists >>= 1) {
       if (warp < lists / 2) {
@@ -149,21 +252,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(
         unsigned long long m[2];
         m[0] = A[lane] > B[63 - lane] ? A[lane] : B[63 - lane];
         m[1] = A[32 + lane] > B[31 - lane] ? A[32 + lane] : B[31 - lane];
-        // m is bitonic: half-cleaner stages 32, 16, ..., 1 sort it descending
-        {
-          const unsigned long long a = m[0], b = m[1];
-          m[0] = a > b ? a : b;
-          m[1] = a > b ? b : a;
-        }
-#pragma unroll
-        for (int j = 16; j > 0; j >>= 1) {
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const unsigned long long o = shfl_xor_u64(m[r], j);
-            const bool lower = (lane & j) == 0;
-            m[r] = lower ? (m[r] > o ? m[r] : o) : (m[r] < o ? m[r] : o);
-          }
-        }
+        warp_bitonic_merge64_desc(m, lane);
         unsigned long long* D = buf[cur ^ 1] + warp * 64;
         D[lane] = m[0];
         D[32 + lane] = m[1];

@@ -272,21 +272,23 @@ def test_topk_ties_and_ragged_candidates(seed):
 
 @pytest.mark.parametrize("seed", [0, 1])
 def test_topk_small_selection_path(seed):
-    """k <= 64 from at most 2048 candidates (the register-sort path) at its
-    edges: 1, 63, 64, 65, 2047 and 2048 candidates, one sequence just past the
-    path (2049, the radix select), heavy ties, k_per_seq 0, 1, 63 and 64."""
+    """k <= 64 from at most 8192 candidates (the register-sort path) at its
+    edges: 1, 63, 64, 65, 127-129, 2047-2049 and 8192 candidates (one to four
+    blocks of 128 per warp), one sequence just past the path (8193, the radix
+    select over unstaged keys), heavy ties, k_per_seq 0, 1, 63 and 64."""
     rng = np.random.default_rng(100 + seed)
-    n_cand = np.array([1, 63, 64, 65, 500, 2047, 2048, 2049, 1536, 700], np.int64)
+    n_cand = np.array([1, 63, 64, 65, 127, 128, 129, 2047, 2048, 2049, 8192, 8193, 1536, 700],
+                      np.int64)
     B = len(n_cand)
     L = n_cand + rng.integers(0, 40, B)
     cu = np.zeros(B + 1, np.int32)
     cu[1:] = np.cumsum(L)
     imp = (rng.integers(0, 12, cu[-1]) * 0.25).astype(np.float32)  # many equal scores
-    imp[cu[9]:cu[10]] = 0.5  # one sequence of ties only
+    imp[cu[13]:cu[14]] = 0.5  # one sequence of ties only
     lo = np.array([rng.integers(0, l - c + 1) for l, c in zip(L, n_cand)], np.int32)
     hi = (lo + n_cand).astype(np.int32)
     K = 64
-    kb = np.array([1, 63, 64, 64, 17, 64, 64, 64, 0, 64], np.int32)
+    kb = np.array([1, 63, 64, 64, 64, 64, 64, 17, 64, 64, 64, 64, 0, 64], np.int32)
     inp = workloads.generate("tiny_fp32")
     dev = tl.upload(inp)
     layer = tl.make_layer(inp, dev["w"], max_topk=K, max_total_k=int(cu[-1]), max_pos=int(L.max()),
