@@ -185,10 +185,13 @@ FC_API fc_status fc_topk_tracked(fc_handle* h, void* stream, int batch, int tota
  * The call returns once the work is queued; it does not wait for the GPU.
  * Two handle-owned copy streams and two sets of device staging buffers let
  * the input copy of one call and the output copy of the previous call run
- * while the kernels of the current call run on `stream`.  Host input buffers
- * must stay unchanged, and out / tracked must not be read, until the caller
- * has called fc_host_sync(h, stream) and `stream` has reached that point
- * (e.g. cudaStreamSynchronize).  Page-locked host memory makes the copies
+ * while the kernels of the current call run on `stream`.  q_pos, the two
+ * cu_seqlens, cand_lo, cand_hi and k_per_seq are read during the call
+ * (gathered into a handle-owned pinned block that is copied as one; the call
+ * waits on the host if that block's copy from two calls earlier is still
+ * running); x must stay unchanged, and out / tracked must not be read, until
+ * the caller has called fc_host_sync(h, stream) and `stream` has reached that
+ * point (e.g. cudaStreamSynchronize).  Page-locked host memory makes the copies
  * asynchronous; pageable memory is accepted but serialises the copies with
  * the host.  The first call allocates the staging buffers (two copies of x,
  * the small arrays, out and tracked, sized from the config) and the copy

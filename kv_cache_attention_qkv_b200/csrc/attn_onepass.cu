@@ -526,8 +526,7 @@ cudaError_t launch_attn_onepass(const fc_handle* h, cudaStream_t st, const CUten
   p.max_fb = h->ws.max_items;
   p.err = h->ws.err;
   const size_t smem = attn_onepass_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(attn_onepass_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = smem_attr(attn_onepass_kernel, smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl_if(h->pdl, attn_onepass_kernel, dim3(h->num_sms), dim3(THREADS), smem, st, h->tm_q, tm_k,
                  tm_v, p);

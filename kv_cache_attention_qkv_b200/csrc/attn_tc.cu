@@ -768,8 +768,7 @@ cudaError_t launch_attn_tc(const fc_handle* h, cudaStream_t st, const StepShape&
   // mode 0 both passes, 1 pass 1 only (row statistics), 2 pass 2 only
   auto kernel = mode == 1 ? attn_tc_kernel<1> : mode == 2 ? attn_tc_kernel<2> : attn_tc_kernel<0>;
   const size_t smem = attn_tc_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = smem_attr(kernel, smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl_if(h->pdl, kernel, dim3(h->num_sms), dim3(THREADS), smem, st, h->tm_q, tm_k, tm_v, p);
   if (e != cudaSuccess) return e;

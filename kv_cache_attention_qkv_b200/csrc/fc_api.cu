@@ -9,6 +9,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -69,6 +70,15 @@ struct ProfScope {
   }
 };
 
+// Kernels whose shared-memory attribute is set, per device and size.
+struct SmemAttrDone {
+  const void* fn;
+  int device;
+  size_t bytes;
+};
+std::mutex g_smem_attr_mu;
+std::vector<SmemAttrDone> g_smem_attr_done;
+
 // Record a failed CUDA call of a step (slot: the kernel being launched, or -1)
 // and return FC_ERR_CUDA.
 fc_status cuda_fail(fc_handle* h, int slot, cudaError_t e) {
@@ -80,6 +90,22 @@ fc_status cuda_fail(fc_handle* h, int slot, cudaError_t e) {
 }  // namespace
 
 namespace fc {
+
+cudaError_t smem_attr_once(const void* fn, size_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lk(g_smem_attr_mu);
+    for (const SmemAttrDone& d : g_smem_attr_done)
+      if (d.fn == fn && d.device == dev && d.bytes >= bytes) return cudaSuccess;
+  }
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(g_smem_attr_mu);
+  g_smem_attr_done.push_back({fn, dev, bytes});
+  return cudaSuccess;
+}
 
 // 2-D bf16 tensor map over a row-major [rows, cols] array, box [box_rows,
 // box_cols], 128-byte swizzle (box_cols * 2 must be 128).

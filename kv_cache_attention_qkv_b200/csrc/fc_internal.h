@@ -102,6 +102,7 @@ struct HostPipe {
   cudaStream_t s_h2d = nullptr, s_d2h = nullptr;
   void* x[2] = {nullptr, nullptr};        // [max_total_q, hidden] dtype
   int32_t* small[2] = {nullptr, nullptr}; // q_pos | cu_q | cu_k | lo | hi | k_per_seq
+  int32_t* small_h[2] = {nullptr, nullptr};  // pinned host copy of that block (one DMA per call)
   void* out[2] = {nullptr, nullptr};      // [max_total_q, H, d] dtype
   int32_t* tracked[2] = {nullptr, nullptr};  // [max_batch, max_topk]
   float* importance = nullptr;            // [max_total_k]
@@ -194,6 +195,14 @@ template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t st, Args... args) {
   return launch_pdl_if(true, kernel, grid, block, smem, st, args...);
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize, bytes) for `fn`, once per
+// kernel, device and size: the runtime call costs host time at every launch.
+cudaError_t smem_attr_once(const void* fn, size_t bytes);
+template <typename... A>
+inline cudaError_t smem_attr(void (*fn)(A...), size_t bytes) {
+  return smem_attr_once(reinterpret_cast<const void*>(fn), bytes);
 }
 
 // ---- launchers (each returns the CUDA error of its launch) -----------------

@@ -340,8 +340,7 @@ cudaError_t launch_gemm_tc(int num_sms, cudaStream_t st, const CUtensorMap& tm_a
                                                         (48ull << 20) / a_block_bytes));
   if (p.num_tiles == 0) return cudaSuccess;
   const size_t smem = gemm_tc_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = smem_attr(gemm_tc_kernel, smem);
   if (e != cudaSuccess) return e;
   int pairs = num_sms / 2;
   if (p.num_tiles < pairs) pairs = p.num_tiles;

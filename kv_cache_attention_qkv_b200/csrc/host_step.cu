@@ -7,6 +7,8 @@
 // (the last reader of that set's out / tracked); the output copy (s_d2h) waits
 // for the kernels.  So the input copy of call n+1 and the output copy of call
 // n-1 run while the kernels of call n run.
+#include <string.h>
+
 #include "fc_internal.h"
 
 namespace {
@@ -54,6 +56,8 @@ fc_status init_pipe(fc_handle* h) {
   for (int s = 0; s < 2 && ok; ++s) {
     ok = cudaMalloc(&p.x[s], (size_t)c.max_total_q * c.hidden * es) == cudaSuccess &&
          cudaMalloc(&p.small[s], small_layout(c).total * sizeof(int32_t)) == cudaSuccess &&
+         cudaHostAlloc(&p.small_h[s], small_layout(c).total * sizeof(int32_t),
+                       cudaHostAllocDefault) == cudaSuccess &&
          cudaMalloc(&p.out[s], (size_t)c.max_total_q * c.n_heads * c.head_dim * es) ==
              cudaSuccess &&
          cudaMalloc(&p.tracked[s], (size_t)c.max_batch * topk * sizeof(int32_t)) == cudaSuccess &&
@@ -81,6 +85,7 @@ void free_host_pipe(fc_handle* h) {
   for (int s = 0; s < 2; ++s) {
     if (p.x[s]) cudaFree(p.x[s]);
     if (p.small[s]) cudaFree(p.small[s]);
+    if (p.small_h[s]) cudaFreeHost(p.small_h[s]);
     if (p.out[s]) cudaFree(p.out[s]);
     if (p.tracked[s]) cudaFree(p.tracked[s]);
     if (p.h2d_done[s]) cudaEventDestroy(p.h2d_done[s]);
@@ -134,12 +139,21 @@ fc_status fc_step_host(fc_handle* h, void* stream, int batch, const void* x, con
       e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, p.s_h2d);
   };
   h2d(p.x[s], x, x_bytes);
-  h2d(sm + L.q_pos, q_pos, (size_t)total_q * sizeof(int32_t));
-  h2d(sm + L.cu_q, cu_seqlens_q, (size_t)(batch + 1) * sizeof(int32_t));
-  h2d(sm + L.cu_k, cu_seqlens_k, (size_t)(batch + 1) * sizeof(int32_t));
-  h2d(sm + L.lo, cand_lo, (size_t)batch * sizeof(int32_t));
-  h2d(sm + L.hi, cand_hi, (size_t)batch * sizeof(int32_t));
-  if (k_per_seq) h2d(sm + L.kps, k_per_seq, (size_t)batch * sizeof(int32_t));
+  // the small arrays are gathered on the host into this set's pinned block
+  // (read now, at the call) and moved in one copy: one driver call instead of
+  // six.  The block's previous copy (call n-2) finished long ago as a rule;
+  // the host waits for it if not.
+  if (e == cudaSuccess && reuse) e = cudaEventSynchronize(p.h2d_done[s]);
+  if (e == cudaSuccess) {
+    int32_t* hb = p.small_h[s];
+    memcpy(hb + L.q_pos, q_pos, (size_t)total_q * sizeof(int32_t));
+    memcpy(hb + L.cu_q, cu_seqlens_q, (size_t)(batch + 1) * sizeof(int32_t));
+    memcpy(hb + L.cu_k, cu_seqlens_k, (size_t)(batch + 1) * sizeof(int32_t));
+    memcpy(hb + L.lo, cand_lo, (size_t)batch * sizeof(int32_t));
+    memcpy(hb + L.hi, cand_hi, (size_t)batch * sizeof(int32_t));
+    if (k_per_seq) memcpy(hb + L.kps, k_per_seq, (size_t)batch * sizeof(int32_t));
+    h2d(sm, hb, (k_per_seq ? L.kps + (size_t)batch : L.kps) * sizeof(int32_t));
+  }
   fc::prof_end(h, p.s_h2d, rec_in);
   if (e == cudaSuccess) e = cudaEventRecord(p.h2d_done[s], p.s_h2d);
   // ---- kernels on the caller's stream

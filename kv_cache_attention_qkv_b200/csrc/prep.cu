@@ -233,8 +233,7 @@ cudaError_t launch_prep(const fc_handle* h, cudaStream_t st, const StepShape& s,
                         int qtile, int long_tiles, int split_sms, int split_min_tiles) {
   size_t smem = prep_smem_bytes(h->cfg.max_pos, h->cfg.max_batch);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = smem_attr(prep_kernel, smem);
     if (e != cudaSuccess) return e;
   }
   prep_kernel<<<s.B + 1, 512, smem, st>>>(s, q_pos, cu_q, cu_k, h->ws.row_dst, h->ws.items,

@@ -361,8 +361,7 @@ cudaError_t launch_qkv_splitk(const fc_handle* h, cudaStream_t st, const StepSha
   p.q_scale = (float)(1.4426950408889634 / sqrt((double)HD));
   p.err = h->ws.err;
   const size_t smem = qkv_splitk_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(qkv_splitk_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = smem_attr(qkv_splitk_kernel, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];

@@ -362,8 +362,7 @@ cudaError_t launch_qkv_tc(const fc_handle* h, cudaStream_t st, const StepShape& 
   p.q_scale = (float)(1.4426950408889634 / sqrt((double)HD));
   p.err = h->ws.err;
   const size_t smem = qkv_tc_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(qkv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = smem_attr(qkv_tc_kernel, smem);
   if (e != cudaSuccess) return e;
   int pairs = h->num_sms / 2;
   if (p.num_tiles < pairs) pairs = p.num_tiles;
