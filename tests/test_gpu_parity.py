@@ -132,6 +132,29 @@ def test_split_attention_agrees_with_unsplit(name):
             np.testing.assert_array_equal(a["tracked"], b["tracked"])
 
 
+def test_split_attention_repeated_on_one_handle():
+    """Consecutive split steps on one handle (the per-item counters of the last
+    entry are reset by the step that used them) give identical results, with
+    and without importance in between."""
+    inp = workloads.generate("small_longcache")
+    dev = tl.upload(inp)
+    layer = tl.make_layer(inp, dev["w"])
+    layer.set_attn_split("always")
+    ref = tl.run_oracle(inp)
+    first = None
+    for imp in (True, False, True, True):
+        g = tl.run_gpu(inp, layer=layer, dev=dev, want_importance=imp)
+        assert g["err"] == 0
+        tl.compare_step(inp, g, ref, range(inp.batch))
+        if imp:
+            if first is None:
+                first = g
+            else:
+                assert np.array_equal(g["out"], first["out"])
+                assert np.array_equal(g["importance"], first["importance"])
+                np.testing.assert_array_equal(g["tracked"], first["tracked"])
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("name,seqs", [("sweep_b1_m128_L8192", [0]), ("sweep_b2_m128_L8192", [0, 1]),
                                        ("sweep_b1_m128_L1536", [0]), ("sweep_b2_m256_L8192", [0, 1])])
