@@ -235,12 +235,14 @@ FC_API fc_status fc_selftest_wait_timeout(fc_handle* h, void* stream, int limit_
 /*
  * fc_last_step_work — how the attention work of the handle's last fc_step was
  * split (waits for the stream of the last call):
- *   items           work items, one per (sequence, head, query tile);
+ *   items           work items, one per (sequence, head, query tile), or, in
+ *                   a small-batch step split over the SMs (FC_OPT_ATTN_SPLIT),
+ *                   one per work entry (an item's run of key tiles);
  *   two_pass_items  items given to the two-pass attention kernel from the
  *                   start: all of them when the step asked for importance (it
  *                   needs every row's final normaliser before the column sums,
- *                   so that kernel scans K twice), none otherwise (bf16 tensor-
- *                   core path; 0 on the CUDA-core path);
+ *                   so that kernel scans K twice) or was split, none otherwise
+ *                   (bf16 tensor-core path; 0 on the CUDA-core path);
  *   handed_over     items of a step without importance that the one-pass
  *                   kernel handed to the two-pass kernel because a score
  *                   exceeded its row's reference (the maximum over the item's
