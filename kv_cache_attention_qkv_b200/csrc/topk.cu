@@ -15,13 +15,13 @@
 //
 // Small selections (k <= 64 from at most 8192 candidates, the usual case) take
 // a path with five block barriers instead of about forty: each of the 16 warps
-// takes a run of up to 512 candidates in blocks of 128 and keeps the 64
-// largest seen so far, in registers, as composite keys score << 32 | ~position
-// (so ties go to the lower position).  The first block is sorted by a bitonic
-// network as wide as the run needs (32, 64 or 128 keys); of each later block
-// only the keys above the current 64th largest can enter, and when there are
-// at most 32 of them (the usual case once the running list has filled) they
-// are packed into one register and sorted alone.  The warps' lists are then
+// takes a run of up to 512 candidates in blocks of 64 and keeps the 64 largest
+// seen so far, in registers, as composite keys score << 32 | ~position (so
+// ties go to the lower position).  The first block is sorted by a bitonic
+// network as wide as the run needs (32 or 64 keys); of each later block only
+// the keys above the current 64th largest can enter, and when there are at
+// most 32 of them (the usual case once the running list has filled) they are
+// packed into one register and sorted alone.  The warps' lists are then
 // merged pairwise in four rounds.  Merging two sorted
 // lists of 64: their elementwise maxima against the other list reversed are
 // the 64 largest and form a bitonic sequence, sorted by one half-cleaner
@@ -191,33 +191,28 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(
       run[0] = m[0];
       run[1] = m[1];
     };
-    // first block: a network only as wide as the warp's run needs
+    // first block of 64: a network only as wide as the warp's run needs
     if (per <= 32) {
       unsigned long long v[1] = {ckey(lane)};
       warp_bitonic_desc<1>(v, lane);
       run[0] = v[0];
-    } else if (per <= 64) {
+    } else {
       unsigned long long v[2] = {ckey(lane), ckey(32 + lane)};
       warp_bitonic_desc<2>(v, lane);
       run[0] = v[0];
       run[1] = v[1];
-    } else {
-      unsigned long long v[4] = {ckey(lane), ckey(32 + lane), ckey(64 + lane), ckey(96 + lane)};
-      warp_bitonic_desc<4>(v, lane);
-      run[0] = v[0];
-      run[1] = v[1];
     }
-    // later blocks: only keys above the current 64th largest can enter; up to
-    // 32 of them are packed into one register (through this warp's slice of
-    // sel) and sorted alone
+    // later blocks of 64: only keys above the current 64th largest can enter;
+    // up to 32 of them are packed into one register (through this warp's
+    // slice of sel) and sorted alone, more are sorted as the block of 64
     unsigned long long* pack = sel + warp * 64;
-    for (int b0 = 128; b0 < per; b0 += 128) {
+    for (int b0 = 64; b0 < per; b0 += 64) {
       const unsigned long long tau = shfl_idx_u64(run[1], 31);  // the 64th largest so far
-      unsigned long long v[4];
-      uint32_t bal[4];
+      unsigned long long v[2];
+      uint32_t bal[2];
       int cnt = 0;
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
+      for (int r = 0; r < 2; ++r) {
         v[r] = ckey(b0 + 32 * r + lane);
         bal[r] = __ballot_sync(0xffffffffu, v[r] > tau);
         cnt += __popc(bal[r]);
@@ -226,7 +221,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(
       if (cnt <= 32) {
         int off = 0;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int r = 0; r < 2; ++r) {
           if (v[r] > tau) pack[off + __popc(bal[r] & ((1u << lane) - 1u))] = v[r];
           off += __popc(bal[r]);
         }
@@ -236,7 +231,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(
         warp_bitonic_desc<1>(x, lane);
         merge_into_run(x[0], 0ull);
       } else {
-        warp_bitonic_desc<4>(v, lane);
+        warp_bitonic_desc<2>(v, lane);
         merge_into_run(v[0], v[1]);
       }
     }
