@@ -21,8 +21,10 @@
 // network as wide as the run needs (32 or 64 keys); of each later block only
 // the keys above the current 64th largest can enter, and when there are at
 // most 32 of them (the usual case once the running list has filled) they are
-// packed into one register and sorted alone.  The warps' lists are then
-// merged pairwise in four rounds.  Merging two sorted
+// packed into one register and sorted alone.  Lists longer than 128 per warp
+// first merge every warp's first 64 keys: the 64th largest of those bounds
+// the answer from below, and only later keys above it are gathered and
+// sorted.  The warps' lists are then merged pairwise in four rounds.  Merging two sorted
 // lists of 64: their elementwise maxima against the other list reversed are
 // the 64 largest and form a bitonic sequence, sorted by one half-cleaner
 // network.
@@ -202,11 +204,83 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(
       run[0] = v[0];
       run[1] = v[1];
     }
-    // later blocks of 64: only keys above the current 64th largest can enter;
-    // up to 32 of them are packed into one register (through this warp's
-    // slice of sel) and sorted alone, more are sorted as the block of 64
     unsigned long long* pack = sel + warp * 64;
-    for (int b0 = 64; b0 < per; b0 += 64) {
+    // the 64 largest of the 16 lists in sel (list w at w * 64), merged
+    // pairwise in four rounds into list 0, in place: in round r, warp w merges
+    // lists 2^(r+1) w and 2^(r+1) w + 2^r into the first of them (each list is
+    // read by one warp, and each lane reads the elements it writes first)
+    auto merge_lists = [&]() {
+      for (int stride = 1; stride < TK_THREADS / 32; stride <<= 1) {
+        if (2 * stride * warp < TK_THREADS / 32) {
+          unsigned long long* A = sel + (2 * stride * warp) * 64;
+          const unsigned long long* B = A + stride * 64;
+          unsigned long long m[2];
+          m[0] = A[lane] > B[63 - lane] ? A[lane] : B[63 - lane];
+          m[1] = A[32 + lane] > B[31 - lane] ? A[32 + lane] : B[31 - lane];
+          warp_bitonic_merge64_desc(m, lane);
+          A[lane] = m[0];
+          A[32 + lane] = m[1];
+        }
+        __syncthreads();
+      }
+    };
+    if (per > 128) {
+      // Long lists: the 64 largest of all warps' first blocks (G) bound the
+      // answer from below: a later key at or below G's 64th cannot be
+      // selected.  Each warp gathers its later keys above that (and above its
+      // own running 64th largest) and sorts them 64 at a time; warp 0 adds G.
+      pack[lane] = run[0];
+      pack[32 + lane] = run[1];
+      __syncthreads();
+      merge_lists();
+      const unsigned long long tau_g = sel[63];
+      unsigned long long g[2] = {0ull, 0ull};
+      if (warp == 0) {
+        g[0] = sel[lane];
+        g[1] = sel[32 + lane];
+      }
+      __syncthreads();  // G is read before the lists are reused as packs
+      run[0] = run[1] = 0ull;
+      int pcount = 0;
+      auto flush = [&]() {
+        unsigned long long x[2] = {lane < pcount ? pack[lane] : 0ull,
+                                   32 + lane < pcount ? pack[32 + lane] : 0ull};
+        __syncwarp();
+        warp_bitonic_desc<2>(x, lane);
+        merge_into_run(x[0], x[1]);
+        pcount = 0;
+      };
+      for (int b0 = 64; b0 < per; b0 += 64) {
+        unsigned long long thr = shfl_idx_u64(run[1], 31);
+        if (thr < tau_g) thr = tau_g;
+        unsigned long long v[2];
+        uint32_t bal[2];
+        int cnt = 0;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          v[r] = ckey(b0 + 32 * r + lane);
+          bal[r] = __ballot_sync(0xffffffffu, v[r] > thr);
+          cnt += __popc(bal[r]);
+        }
+        if (cnt == 0) continue;
+        if (pcount + cnt > 64) flush();
+        int off = pcount;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          if (v[r] > thr) pack[off + __popc(bal[r] & ((1u << lane) - 1u))] = v[r];
+          off += __popc(bal[r]);
+        }
+        pcount = off;
+        __syncwarp();
+      }
+      if (pcount > 0) flush();
+      if (warp == 0) merge_into_run(g[0], g[1]);
+    }
+    // later blocks of 64 (lists of at most 128 per warp): only keys above the
+    // current 64th largest can enter; up to 32 of them are packed into one
+    // register (through this warp's slice of sel) and sorted alone, more are
+    // sorted as the block of 64
+    for (int b0 = 64; b0 < per && per <= 128; b0 += 64) {
       const unsigned long long tau = shfl_idx_u64(run[1], 31);  // the 64th largest so far
       unsigned long long v[2];
       uint32_t bal[2];
@@ -235,28 +309,13 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(
         merge_into_run(v[0], v[1]);
       }
     }
-    unsigned long long* buf[2] = {sel, reinterpret_cast<unsigned long long*>(skey)};
-    buf[0][warp * 64 + lane] = run[0];
-    buf[0][warp * 64 + 32 + lane] = run[1];
-    __syncthreads();  // every warp has also finished reading skey (buf[1])
-    int cur = 0;
-    for (int lists = TK_THREADS / 32; lists > 1; lists >>= 1) {
-      if (warp < lists / 2) {
-        const unsigned long long* A = buf[cur] + (2 * warp) * 64;
-        const unsigned long long* B = A + 64;
-        unsigned long long m[2];
-        m[0] = A[lane] > B[63 - lane] ? A[lane] : B[63 - lane];
-        m[1] = A[32 + lane] > B[31 - lane] ? A[32 + lane] : B[31 - lane];
-        warp_bitonic_merge64_desc(m, lane);
-        unsigned long long* D = buf[cur ^ 1] + warp * 64;
-        D[lane] = m[0];
-        D[32 + lane] = m[1];
-      }
-      __syncthreads();
-      cur ^= 1;
-    }
+    __syncwarp();
+    pack[lane] = run[0];
+    pack[32 + lane] = run[1];
+    __syncthreads();
+    merge_lists();
     for (int i = tid; i < k; i += TK_THREADS)
-      row[i] = i < want ? (int32_t)(0xFFFFFFFFu - (uint32_t)(buf[cur][i] & 0xFFFFFFFFull)) : -1;
+      row[i] = i < want ? (int32_t)(0xFFFFFFFFu - (uint32_t)(sel[i] & 0xFFFFFFFFull)) : -1;
     return;
   }
 
